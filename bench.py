@@ -1,0 +1,581 @@
+#!/usr/bin/env python
+"""Benchmark of the NF4 + double-quant QLoRA linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of the 7B-shaped MLP
+workload (gate/up [11008 x 4096] and down [4096 x 11008], X [4096 x in]
+= batch 4 x seq 1024, LoRA r=64 alpha=16): for each projection, blockwise
+NF4 quantization with double-quantized absmax of the fp32 weight, the fused
+forward Y = X W^T + s (X A^T) B^T, the input gradient dX and the adapter
+gradients dA, dB.  All inputs are seeded synthetic tensors resident in HBM.
+The metric is whole-job TFLOP/s (algorithmic FLOPs of the linear algebra,
+the quantize pass counted as zero FLOPs but timed); the decode-sized M=1
+weight-streaming forward is reported beside it as weight-GB/s.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch
+(weak scaling, data parallel); the adapter gradients of each step are
+averaged across ranks with one NCCL all-reduce, the data-parallel exchange
+of LoRA training.  Time is measured on the device with CUDA events between
+barriers and the maximum over ranks is reported.
+
+``--impl reference`` times the CPU oracle (``oracle/``) on the host cores
+instead, on a bounded sample of the same workload per step.
+"""
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "fused NF4 linear TFLOPS (M=4096) and weight-GB/s (M=1) vs B200 roofline"
+UNIT = "TFLOP/s"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "fused_fwd_gemm_7b_mlp.txt")
+
+
+# ---------------------------------------------------------------------------
+# workload description (pure host logic, also used by the CPU tests)
+# ---------------------------------------------------------------------------
+
+PROJECTIONS = ("gate", "up", "down")
+
+
+def linear_flops(m: int, n: int, k: int, r: int) -> dict:
+    """Algorithmic FLOPs of the three linear-algebra rows of the hot path."""
+    fwd = 2 * m * n * k + 2 * m * r * (n + k)             # X W^T, X A^T, T B^T
+    bwd_dx = 2 * m * n * k + 2 * m * r * (n + k)          # dY W^, dY B, U A
+    grads = 2 * m * r * (n + 2 * k) + 2 * m * n * r       # U, T, dA = U^T X, dB = dY^T T
+    return {"fwd": fwd, "bwd_dx": bwd_dx, "grads": grads, "total": fwd + bwd_dx + grads,
+            "fused_fwd_kernel": 2 * m * n * k + 2 * m * n * r}
+
+
+def weight_bytes(n: int, k: int) -> int:
+    """Packed codes + uint8 absmax codes + fp32 group scales."""
+    numel = n * k
+    nb = numel // 64
+    return numel // 2 + nb + 4 * ((nb + 255) // 256)
+
+
+def step_flops(cases) -> int:
+    return sum(linear_flops(c.m, c.n, c.k, c.r)["total"] for c in cases)
+
+
+def load_peaks() -> tuple:
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Maximum of a per-rank float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def allreduce_grads(flat, world: int) -> None:
+    """Average the flat adapter-gradient buffer over ranks (data parallel)."""
+    if world <= 1:
+        return
+    import torch.distributed as dist
+    dist.all_reduce(flat, op=dist.ReduceOp.SUM)
+    flat.div_(world)
+
+
+def profile_traffic(src_digest: str):
+    """DRAM bytes per launch of the fused forward GEMM from the committed ncu
+    summary, or None when that summary was taken on a different kernel source."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            txt = f.read()
+    except OSError:
+        return None
+    digest, traffic = None, None
+    for line in txt.splitlines():
+        if line.startswith("kernel_source_sha256:"):
+            digest = line.split(":", 1)[1].strip()
+        if line.startswith("traffic_bytes_per_launch:"):
+            traffic = float(line.split(":", 1)[1].strip())
+    return traffic if digest == src_digest else None
+
+
+def kernel_source_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("tc_gemm.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "bit_nf4_quantized_qlora_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region (NVML, read-only)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int, interval_s: float = 0.01):
+        self.idx = device_index
+        self.dt = interval_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = None
+            try:                                   # the CUDA device, found by PCI bus id
+                import torch
+                pr = torch.cuda.get_device_properties(device_index)
+                bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            self._reasons_fn = fn
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self._reasons_fn(self.h))
+            except Exception:
+                pass
+            time.sleep(self.dt)
+
+    def __enter__(self):
+        if self.ok:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thr:
+            self._thr.join()
+
+    def summary(self) -> dict:
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [k for k, bit in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def _dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+class Projection:
+    """Device-resident state of one NF4 + LoRA projection of the step."""
+
+    def __init__(self, case, dev, grad_view_a, grad_view_b):
+        import torch
+        from bit_nf4_quantized_qlora_b200 import binding as B
+        self.case = case
+        self.W = case.W().to(dev)
+        self.X = case.X().to(dev)
+        self.dY = case.dY().to(dev)
+        self.A = case.A().to(dev)
+        self.B = case.B().to(dev)
+        n, k, m, r = case.n, case.k, case.m, case.r
+        numel = n * k
+        self.w = B.NF4Weight(torch.empty(numel // 2, dtype=torch.uint8, device=dev),
+                             torch.empty(numel // 64, dtype=torch.uint8, device=dev),
+                             torch.empty(B.n_groups(numel), dtype=torch.float32, device=dev), n, k)
+        self.Y = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
+        self.dX = torch.empty(m, k, dtype=torch.bfloat16, device=dev)
+        self.dA, self.dB = grad_view_a, grad_view_b
+        self.ws_f = torch.empty(B.qlora_workspace_bytes(B.QLORA_OP_FWD, m, n, k, r), dtype=torch.uint8, device=dev)
+        self.ws_b = torch.empty(B.qlora_workspace_bytes(B.QLORA_OP_BWD_DX, m, n, k, r), dtype=torch.uint8, device=dev)
+        self.ws_g = torch.empty(B.qlora_workspace_bytes(B.QLORA_OP_LORA_BWD, m, n, k, r), dtype=torch.uint8,
+                                device=dev)
+
+    def run(self, prof=None):
+        """The hot path of this projection: quantize, fwd, bwd_dx, grads."""
+        from bit_nf4_quantized_qlora_b200 import binding as B
+        c = self.case
+        B.qlora_quantize_nf4_dq(self.W, out=self.w)
+        if prof is not None:
+            B.qlora_set_profile_events(*prof)
+        B.qlora_linear_fwd(self.X, self.w, self.A, self.B, c.r, c.scale, out=self.Y, ws=self.ws_f)
+        if prof is not None:
+            B.qlora_set_profile_events(None, None)
+        B.qlora_linear_bwd_dx(self.dY, self.w, self.A, self.B, c.r, c.scale, out=self.dX, ws=self.ws_b)
+        B.qlora_lora_bwd(self.X, self.dY, self.A, self.B, c.r, c.scale, dA=self.dA, dB=self.dB, ws=self.ws_g)
+
+
+def _grad_buffer(cases, dev):
+    import torch
+    sizes = [c.r * c.k + c.n * c.r for c in cases]
+    flat = torch.zeros(sum(sizes), dtype=torch.bfloat16, device=dev)
+    views, off = [], 0
+    for c in cases:
+        a = flat[off:off + c.r * c.k].view(c.r, c.k)
+        off += c.r * c.k
+        b = flat[off:off + c.n * c.r].view(c.n, c.r)
+        off += c.n * c.r
+        views.append((a, b))
+    return flat, views
+
+
+def _m1_decode(dev, peaks, peak_kind):
+    """Weight-GB/s of the M=1 forward on the 4096x4096 (7B attention) and
+    28672x8192 (70B up-projection) weights: CUDA-graph replays over rotating
+    weight copies whose total size exceeds 2x the L2, so the weights come from
+    HBM on every call."""
+    import torch
+    from bit_nf4_quantized_qlora_b200 import binding as B
+    from bit_nf4_quantized_qlora_b200 import workloads as WL
+    out = {}
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    for name, case in (("attn_proj_4096x4096", WL.attn_proj_7b(1)), ("up_proj_28672x8192", WL.up_proj_70b(1))):
+        wb = weight_bytes(case.n, case.k)
+        copies = max(2, int(2 * l2 // wb) + 1)
+        W = case.W().to(dev)
+        w0 = B.qlora_quantize_nf4_dq(W)
+        del W
+        ws = [w0] + [B.NF4Weight(w0.codes.clone(), w0.absmax_q.clone(), w0.group_scale.clone(), case.n, case.k)
+                     for _ in range(copies - 1)]
+        X = case.X().to(dev)
+        A, Bm = case.A().to(dev), case.B().to(dev)
+        Y = torch.empty(1, case.n, dtype=torch.bfloat16, device=dev)
+        wsp = torch.empty(B.qlora_workspace_bytes(B.QLORA_OP_FWD, 1, case.n, case.k, case.r), dtype=torch.uint8,
+                          device=dev)
+        s = torch.cuda.Stream()
+        with torch.cuda.stream(s):
+            for w in ws:                                   # warm-up outside capture
+                B.qlora_linear_fwd(X, w, A, Bm, case.r, case.scale, out=Y, ws=wsp)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                for w in ws:
+                    B.qlora_linear_fwd(X, w, A, Bm, case.r, case.scale, out=Y, ws=wsp)
+        reps = max(3, int(200e6 // (wb * copies)) + 1)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        t_call = e0.elapsed_time(e1) * 1e-3 / (reps * copies)
+        gbs = (wb + 2 * case.r * (case.n + case.k)) / t_call / 1e9
+        out[name] = {"us_per_call": round(t_call * 1e6, 3), "weight_gbps": round(gbs, 1),
+                     "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4), "peak_kind": peak_kind,
+                     "weight_copies": copies, "cuda_graph": True, "lora_r": case.r}
+        del g, ws, w0
+        torch.cuda.empty_cache()
+    return out
+
+
+def _cpu_baseline(rank: int, world: int):
+    if rank != 0 or world != 1:
+        return None
+    try:
+        return reference_step_sample(rows=48, repeat=1)
+    except Exception as e:  # the oracle is a reported baseline only
+        return {"value": None, "unit": UNIT, "kind": "oracle", "error": str(e)}
+
+
+def run_ours(args):
+    import torch
+    from bit_nf4_quantized_qlora_b200 import binding as B
+    from bit_nf4_quantized_qlora_b200 import workloads as WL
+
+    world, rank, local = _dist_setup()
+    dev = torch.device("cuda", local)
+    B.lib()                                          # fails loudly without the CUDA library
+    peaks, peak_kind = load_peaks()
+    cases = [WL.mlp_7b(p) for p in PROJECTIONS]
+    flat, views = _grad_buffer(cases, dev)
+    projs = [Projection(c, dev, a, b) for c, (a, b) in zip(cases, views)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(prof=None):
+        for i, p in enumerate(projs):
+            p.run(prof[i] if prof is not None else None)
+        allreduce_grads(flat, world)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # Per-launch events for the fused forward GEMM (gate and up share a shape).
+    K = args.steps
+    prof_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in projs]
+               for _ in range(K)]
+    for pair in prof_ev:
+        for a, b in pair:                              # materialise the event handles
+            a.record(stream)
+            b.record(stream)
+    torch.cuda.synchronize()
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = B.qlora_launch_count()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for i in range(K):
+            step(prof_ev[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    launches = B.qlora_launch_count() - launches0
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    elapsed = t0.elapsed_time(t1) * 1e-3
+    elapsed = reduce_max(elapsed, world, dev)
+    dev_err = B.qlora_poll_device_error()
+
+    total_flops = step_flops(cases) * world * K
+    value = total_flops / elapsed / 1e12
+    ms_per_step = elapsed / K * 1e3
+
+    # Live roofline of the dominant kernel: the fused forward GEMM of gate/up.
+    gu = [prof_ev[i][j][0].elapsed_time(prof_ev[i][j][1]) * 1e-3 for i in range(K) for j in (0, 1)]
+    t_launch = sum(gu) / len(gu)
+    f_launch = linear_flops(cases[0].m, cases[0].n, cases[0].k, cases[0].r)["fused_fwd_kernel"]
+    achieved = f_launch / t_launch / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    traffic = profile_traffic(kernel_source_digest())
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "kernel": "tc_kernel fused NF4 dequant + tcgen05 GEMM (forward, 4096x11008x4096, LoRA r=64)",
+                "flops_per_launch": f_launch, "launch_us": round(t_launch * 1e6, 2),
+                "peak_kind": f"{peak_kind} sustained bf16 (cuBLAS, long loop under the power cap)"}
+
+    # End to end through the public API with host buffers.
+    e2e = _e2e(projs, cases, flat, world, dev, stream, max(3, min(K, 10)))
+
+    m1 = _m1_decode(dev, peaks, peak_kind) if rank == 0 else None
+    cpu = _cpu_baseline(rank, world)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "7B-shaped MLP gate/up [11008x4096] + down [4096x11008], NF4 block 64 + "
+                                   "8-bit double-quant per 256 blocks, X bf16 [4096 x in] (batch 4 x seq 1024), "
+                                   "LoRA r=64 alpha=16; step = quantize + fwd + bwd_dx + LoRA grads per projection",
+                       "global_batch": 4 * world, "seq_len": 1024, "parallelism": f"dp{world}",
+                       "l2": "inputs larger than L2 (fp32 weights 541 MB + activations/grads per step)"},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": int(launches),
+            "clocks": clk.summary(),
+            "m1_decode": m1,
+            "device_error_flags": dev_err,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _e2e(projs, cases, flat, world, dev, stream, steps):
+    """Same metric through the binding with pinned host inputs: every step
+    copies X and dY of all projections host->device, runs the step, and
+    copies the adapter gradients device->host."""
+    import torch
+    host_in = [(p.X.cpu().pin_memory(), p.dY.cpu().pin_memory()) for p in projs]
+    host_grad = torch.empty(flat.numel(), dtype=flat.dtype).pin_memory()
+    h2d = sum(x.numel() * x.element_size() + d.numel() * d.element_size() for x, d in host_in)
+    d2h = flat.numel() * flat.element_size()
+
+    def step():
+        for p, (hx, hd) in zip(projs, host_in):
+            p.X.copy_(hx, non_blocking=True)
+            p.dY.copy_(hd, non_blocking=True)
+        for p in projs:
+            p.run()
+        allreduce_grads(flat, world)
+        host_grad.copy_(flat, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    el = reduce_max(t0.elapsed_time(t1) * 1e-3, world, dev)
+    value = step_flops(cases) * world * steps / el / 1e12
+    return {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "steps": steps, "ms_per_step": round(el / steps * 1e3, 3)}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle on the host cores
+# ---------------------------------------------------------------------------
+
+def _cpu_cores() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        blas = [i for i in info if i.get("user_api") == "blas"]
+        if blas:
+            return int(blas[0].get("num_threads", os.cpu_count() or 1))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+_REF_CACHE = {}
+
+
+def _ref_prepare(rows: int):
+    """Untimed set-up of the oracle sample: per projection the fp32 weight,
+    `rows` token rows of X and dY, and A, B as exact fp64 values."""
+    if rows in _REF_CACHE:
+        return _REF_CACHE[rows]
+    import numpy as np
+    import torch
+    from bit_nf4_quantized_qlora_b200 import workloads as WL
+    items = []
+    for p in PROJECTIONS:
+        c = WL.mlp_7b(p)
+        W = c.W().reshape(-1).numpy()
+        X = c.X()[:rows].to(torch.float32).numpy().astype(np.float64)
+        dY = c.dY()[:rows].to(torch.float32).numpy().astype(np.float64)
+        A = c.A().to(torch.float32).numpy().astype(np.float64)
+        Bm = c.B().to(torch.float32).numpy().astype(np.float64)
+        items.append((c, W, X, dY, A, Bm))
+    _REF_CACHE[rows] = items
+    return items
+
+
+def reference_step_sample(rows: int = 8, repeat: int = 1, quant_groups: int = 64) -> dict:
+    """One bounded sample of the step through the oracle: for each projection,
+    quantize + dequantize `quant_groups` groups of 256 blocks of W, dequantize
+    the rest of W once, then fwd, bwd_dx and the adapter gradients for `rows`
+    token rows.  Returns TFLOP/s of the sampled linear algebra."""
+    import numpy as np
+    from oracle import linear, quant
+    items = _ref_prepare(rows)
+    flops = 0
+    t_total = 0.0
+    for _ in range(repeat):
+        for c, W, X, dY, A, Bm in items:
+            t = time.perf_counter()
+            sample = W[:quant_groups * 16384]
+            p, q, S, _ = quant.quantize_nf4_dq(sample)
+            quant.dequant_bf16_values(p, q, S)
+            t_q = time.perf_counter() - t
+            key = ("what", c.name)
+            if key not in _REF_CACHE:
+                pw, qw, sw, _ = quant.quantize_nf4_dq(W)
+                _REF_CACHE[key] = quant.dequant_bf16_values(pw, qw, sw).reshape(c.n, c.k)
+            W_hat = _REF_CACHE[key]
+            t = time.perf_counter()
+            linear.fwd(X, W_hat, A, Bm, c.scale)
+            linear.bwd_dx(dY, W_hat, A, Bm, c.scale)
+            linear.lora_grads(X, dY, A, Bm, c.scale)
+            t_total += time.perf_counter() - t + t_q
+            flops += linear_flops(rows, c.n, c.k, c.r)["total"]
+    value = flops / t_total / 1e12
+    return {"value": value, "unit": UNIT, "cores": _cpu_cores(), "kind": "oracle",
+            "sample": f"per projection (gate, up, down): oracle quantize+dequantize of {quant_groups} groups "
+                      f"({quant_groups * 16384} weights) and fwd + bwd_dx + LoRA grads in fp64 for {rows} of the "
+                      f"4096 token rows (W^ dequantized once, untimed)",
+            "seconds": round(t_total, 3)}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return                                          # only rank 0 runs the oracle
+    rows = 8
+    _ref_prepare(rows)
+    for _ in range(args.warmup):
+        reference_step_sample(rows=rows)
+    t = time.perf_counter()
+    vals = [reference_step_sample(rows=rows) for _ in range(args.steps)]
+    el = time.perf_counter() - t
+    value = sum(v["value"] for v in vals) / len(vals)
+    sample = vals[0]
+    line = {
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(el / max(1, args.steps) * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": "7B-shaped MLP gate/up [11008x4096] + down [4096x11008], NF4 block 64 + 8-bit "
+                               "double-quant per 256 blocks, LoRA r=64 alpha=16; oracle sample per step",
+                   "global_batch": 4, "seq_len": 1024, "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": sample["cores"], "kind": "oracle",
+                         "sample": sample["sample"]},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

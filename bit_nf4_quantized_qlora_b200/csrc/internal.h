@@ -1,0 +1,70 @@
+// Host-side declarations shared by the translation units of libqlora.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "types.h"
+
+namespace qlora {
+
+// The library's own NF4 codebook and midpoints (derived once at load time).
+const Nf4Tables &nf4_tables();
+
+// Device error word (bounded waits that gave up); one per device.
+unsigned *device_error_word();
+
+// Process-wide count of kernel launches (see qlora_launch_count).
+void count_launches(int n);
+
+// --- launchers (all asynchronous on `stream`; return cudaError_t) --------
+
+cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q,
+                            float *group_scale, float *absmax_fp32, cudaStream_t stream);
+
+cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *absmax_q, const float *group_scale,
+                           int64_t numel, uint16_t *out, cudaStream_t stream);
+
+// T[m x r] = bf16(scale * X[m x k] . A[r x k]^T) for small m (m <= 16).
+cudaError_t launch_lora_proj_small(const uint16_t *X, int64_t m, int64_t k, const uint16_t *A,
+                                   int32_t r, float scale, uint16_t *T, cudaStream_t stream);
+
+// Y[m x n] = bf16(X . W^T + T . B^T) for m <= 16 (weight-streaming kernel).
+cudaError_t launch_gemv_fwd(const uint16_t *X, int64_t m, const uint8_t *codes,
+                            const uint8_t *absmax_q, const float *group_scale, int64_t n, int64_t k,
+                            const uint16_t *T, const uint16_t *B, int32_t r, uint16_t *Y,
+                            cudaStream_t stream);
+
+// tcgen05 paths -------------------------------------------------------------
+
+struct WeightView {
+  const uint8_t *codes;
+  const uint8_t *absmax_q;
+  const float *group_scale;
+  int64_t n, k;
+};
+
+// Y = bf16(X . W^T + T . B^T); T may be null (no adapter).
+cudaError_t tc_fwd(const uint16_t *X, int64_t m, const WeightView &w, const uint16_t *T,
+                   const uint16_t *B, int32_t r, uint16_t *Y, cudaStream_t stream);
+
+// dX = bf16(dY . W^ + U . A); U may be null.
+cudaError_t tc_bwd_dx(const uint16_t *dY, int64_t m, const WeightView &w, const uint16_t *U,
+                      const uint16_t *A, int32_t r, uint16_t *dX, cudaStream_t stream);
+
+// out[m x r] = bf16(scale * L[m x kc] . R^T) with R given as [r x kc] (k-major).
+cudaError_t tc_proj_kmajor(const uint16_t *L, int64_t m, int64_t kc, const uint16_t *R, int32_t r,
+                           float scale, uint16_t *out, cudaStream_t stream);
+
+// out[m x r] = bf16(scale * L[m x kc] . R) with R given as [kc x r] (r contiguous).
+cudaError_t tc_proj_mnmajor(const uint16_t *L, int64_t m, int64_t kc, const uint16_t *R, int32_t r,
+                            float scale, uint16_t *out, cudaStream_t stream);
+
+// out = bf16(Lt^T . R): Lt [mc x p] (p contiguous), R [mc x r] (r contiguous),
+// contraction over mc; result [p x r] stored row-major (transposed == false)
+// or as [r x p] (transposed == true).
+cudaError_t tc_tn_skinny(const uint16_t *Lt, int64_t mc, int64_t p, const uint16_t *R, int32_t r,
+                         uint16_t *out, bool transposed, cudaStream_t stream);
+
+}  // namespace qlora

@@ -1,0 +1,613 @@
+// tcgen05 / TMEM GEMMs for the QLoRA linear layer on sm_100a.
+//
+// One kernel template covers every dense contraction of the layer:
+//
+//   fused forward     D = X . W^T   (+ T . B^T as extra k-steps)
+//   fused bwd_dx      D = dY . W^   (+ U . A   as extra k-steps)
+//   skinny products   T = s X A^T, U = s dY B, dA^T = X^T U, dB = dY^T T
+//
+// "QLoRA and Quantized Training", The idea: compute happens in bf16, each block
+// is dequantized, used in a matrix multiply and discarded; "A 65B fine-tune on
+// the GPU you already have", figure 2: dequantized block by block to bf16 just
+// long enough to multiply.  Here the NF4 weight never exists in bf16 outside
+// shared memory: TMA stages the packed codes of one k-step (one NF4 block per
+// weight row) into shared memory, eight dequant warps expand them into a
+// 128-byte-swizzled bf16 tile, and one thread issues tcgen05.mma on it with
+// the fp32 accumulator in tensor memory.
+//
+// Warp roles (one CTA per output tile, 1 CTA per SM):
+//   warp 0      TMA producer (A operand, packed codes or B operand)
+//   warp 1      TMEM allocator and single-thread MMA issuer
+//   warps 2..   dequant producers during the main loop (NF4 modes), then the
+//               epilogue: tcgen05.ld -> scale -> bf16 -> global
+// Stages are guarded by mbarriers: full_a (TMA bytes landed), full_b (dequant
+// warps wrote the B tile), empty (the MMAs reading the stage completed, via
+// tcgen05.commit), acc (all MMAs done).  Every wait is bounded in time: on a
+// timeout a flag is set in the caller-visible error word and the roles drain
+// and exit; no kernel traps.
+//
+// Shared-memory operand layouts (SWIZZLE_128B, 1024-byte aligned atoms):
+//   K-major tile  [rows x 64] bf16: row r at r*128, 16-byte chunk c stored at
+//                 chunk c ^ (r % 8)             (LBO 16 B, SBO 1024 B)
+//   MN-major tile [64 k-rows x 64*j cols]: slab j (64 columns) at j*8192, k-row
+//                 at 128 B pitch, same swizzle    (LBO 8192 B, SBO 1024 B)
+// One NF4 block (64 consecutive weights of a row) is one 128-byte swizzled
+// row in both layouts, so the forward (weight rows are MMA N, K-major) and the
+// input gradient (weight rows are the contraction, MN-major) share the
+// dequant routine and differ only in which (row, block) lands in which row.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace qlora {
+namespace {
+
+constexpr int kBK = 64;                       // k-step: 64 bf16 = one swizzle row
+constexpr uint32_t kASub = 128u * kBK * 2u;   // 16 KB: one 128-row A tile
+
+struct __align__(64) TcParams {
+  CUtensorMap tmA;      // main A operand
+  CUtensorMap tmB;      // main B operand (bf16 modes)
+  CUtensorMap tmCodes;  // packed codes viewed as [rows x bytes] (NF4 modes)
+  CUtensorMap tmA2;     // adapter A operand (extra k-steps)
+  CUtensorMap tmB2;     // adapter B operand (extra k-steps)
+  const uint8_t *absmax_q;
+  const float *group_scale;
+  uint16_t *out;
+  unsigned *err;
+  int64_t w_n, w_k;     // weight shape (NF4 modes)
+  int64_t out_ld;
+  int out_rows, out_cols;
+  int num_main, num_lora;
+  float alpha;
+  Nf4Tables tab;
+};
+
+// ---- PTX wrappers --------------------------------------------------------
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint64_t *bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((addr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(lbo >> 4) << 16) |
+         (static_cast<uint64_t>(sbo >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// kind::f16 instruction descriptor: bf16 x bf16 -> fp32, M = 128.
+__host__ __device__ constexpr uint32_t make_idesc(int n, bool a_mn, bool b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, const uint32_t (&v)[4]) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
+               : "memory");
+}
+
+// ---- compile-time configuration -------------------------------------------
+
+template <int BN_, int MSUB_, bool A_MN_, bool B_NF4_, bool B_MN_, bool OUT_T_>
+struct Cfg {
+  static constexpr int BN = BN_;
+  static constexpr int MSUB = MSUB_;
+  static constexpr bool A_MN = A_MN_;
+  static constexpr bool B_NF4 = B_NF4_;
+  static constexpr bool B_MN = B_MN_;
+  static constexpr bool OUT_T = OUT_T_;
+  static constexpr int BM = 128 * MSUB;
+  static constexpr uint32_t A_BYTES = kASub * MSUB;
+  static constexpr uint32_t B_BYTES = static_cast<uint32_t>(BN) * kBK * 2u;
+  static constexpr uint32_t CODE_BYTES = B_NF4 ? static_cast<uint32_t>(BN) * 32u : 0u;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + CODE_BYTES;
+  static constexpr int STAGES_RAW = static_cast<int>((224u * 1024u) / STAGE_BYTES);
+  static constexpr int STAGES = STAGES_RAW > 6 ? 6 : STAGES_RAW;
+  static constexpr uint32_t SMEM_BYTES = STAGE_BYTES * STAGES + 1024u;
+  static constexpr int NUM_EPI_WARPS = B_NF4 ? 8 : 4;
+  static constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+  static constexpr uint32_t TMEM_RAW = static_cast<uint32_t>(BN * MSUB);
+  static constexpr uint32_t TMEM_COLS = TMEM_RAW <= 32 ? 32 : TMEM_RAW <= 64 ? 64 : TMEM_RAW <= 128 ? 128 : TMEM_RAW <= 256 ? 256 : 512;
+  static constexpr uint32_t IDESC = make_idesc(BN, A_MN, B_MN);
+  static_assert(STAGES >= 2, "not enough shared memory for two stages");
+  static_assert(!(A_MN && MSUB != 1), "MN-major A supports one 128-row tile");
+  static_assert(!B_NF4 || BN == 256, "NF4 modes use 256-wide tiles (one block per dequant thread)");
+  static_assert(BN % 64 == 0 && BN <= 256, "BN");
+};
+
+template <class C>
+__global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_constant__ TcParams p) {
+  extern __shared__ uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t full_a[C::STAGES];
+  __shared__ __align__(8) uint64_t full_b[C::STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
+  __shared__ __align__(8) uint64_t acc_bar;
+  __shared__ uint32_t tmem_slot;
+
+  const uint32_t raw = smem_u32(dsmem);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_tile = blockIdx.x;
+  const int m_tile = blockIdx.y;
+  const int total = p.num_main + p.num_lora;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full_a[s], 1);
+      mbar_init(&full_b[s], C::B_NF4 ? 8 : 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&acc_bar, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&p.tmA);
+    if (C::B_NF4) tma_prefetch_desc(&p.tmCodes); else tma_prefetch_desc(&p.tmB);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int it = 0; it < total; ++it) {
+        const int s = it % C::STAGES;
+        const uint32_t ph = static_cast<uint32_t>(it / C::STAGES) & 1u;
+        if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, p.err, kErrTimeoutEmpty)) break;
+        const uint32_t a_s = base + static_cast<uint32_t>(s) * C::STAGE_BYTES;
+        const uint32_t b_s = a_s + C::A_BYTES;
+        const uint32_t c_s = b_s + C::B_BYTES;
+        if (it < p.num_main) {
+          mbar_arrive_expect_tx(&full_a[s], C::A_BYTES + (C::B_NF4 ? C::CODE_BYTES : C::B_BYTES));
+          if (!C::A_MN) {
+#pragma unroll
+            for (int h = 0; h < C::MSUB; ++h)
+              tma_load_2d(a_s + h * kASub, &p.tmA, &full_a[s], it * kBK, m_tile * C::BM + h * 128);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              tma_load_2d(a_s + j * 8192u, &p.tmA, &full_a[s], m_tile * 128 + j * 64, it * kBK);
+          }
+          if (C::B_NF4) {
+            if (!C::B_MN) {
+              tma_load_2d(c_s, &p.tmCodes, &full_a[s], it * 32, n_tile * C::BN);
+            } else {
+#pragma unroll
+              for (int j = 0; j < C::BN / 64; ++j)
+                tma_load_2d(c_s + j * 2048u, &p.tmCodes, &full_a[s], n_tile * (C::BN / 2) + 32 * j, it * kBK);
+            }
+          } else {
+            if (!C::B_MN) {
+              tma_load_2d(b_s, &p.tmB, &full_a[s], it * kBK, n_tile * C::BN);
+            } else {
+#pragma unroll
+              for (int j = 0; j < C::BN / 64; ++j)
+                tma_load_2d(b_s + j * 8192u, &p.tmB, &full_a[s], n_tile * C::BN + 64 * j, it * kBK);
+            }
+          }
+        } else {
+          const int l = it - p.num_main;
+          mbar_arrive_expect_tx(&full_a[s], C::A_BYTES + C::B_BYTES);
+#pragma unroll
+          for (int h = 0; h < C::MSUB; ++h)
+            tma_load_2d(a_s + h * kASub, &p.tmA2, &full_a[s], l * kBK, m_tile * C::BM + h * 128);
+          if (!C::B_MN) {
+            tma_load_2d(b_s, &p.tmB2, &full_a[s], l * kBK, n_tile * C::BN);
+          } else {
+#pragma unroll
+            for (int j = 0; j < C::BN / 64; ++j)
+              tma_load_2d(b_s + j * 8192u, &p.tmB2, &full_a[s], n_tile * C::BN + 64 * j, l * kBK);
+          }
+        }
+        ++issued;
+      }
+      // Drain: every issued copy has landed before the CTA may exit.
+      for (int it = issued - C::STAGES < 0 ? 0 : issued - C::STAGES; it < issued; ++it)
+        mbar_wait_bounded(&full_a[it % C::STAGES], static_cast<uint32_t>(it / C::STAGES) & 1u, p.err,
+                          kErrTimeoutDrain);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      for (int it = 0; it < total && ok; ++it) {
+        const int s = it % C::STAGES;
+        const uint32_t ph = static_cast<uint32_t>(it / C::STAGES) & 1u;
+        ok = mbar_wait_bounded(&full_a[s], ph, p.err, kErrTimeoutFullA);
+        if (ok && C::B_NF4) ok = mbar_wait_bounded(&full_b[s], ph, p.err, kErrTimeoutFullB);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t a_s = base + static_cast<uint32_t>(s) * C::STAGE_BYTES;
+        const uint32_t b_s = a_s + C::A_BYTES;
+#pragma unroll
+        for (int h = 0; h < C::MSUB; ++h) {
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = C::A_MN ? smem_desc(a_s + kk * 2048u, 8192u, 1024u)
+                                        : smem_desc(a_s + h * kASub + kk * 32u, 16u, 1024u);
+            const uint64_t bd = C::B_MN ? smem_desc(b_s + kk * 2048u, 8192u, 1024u)
+                                        : smem_desc(b_s + kk * 32u, 16u, 1024u);
+            umma_f16(tmem + static_cast<uint32_t>(h * C::BN), ad, bd, C::IDESC, (it > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(&empty_bar[s]);
+      }
+      if (ok) umma_commit(&acc_bar);
+    }
+  } else {
+    // ------------------------------------------------------------ dequant
+    const int dt = threadIdx.x - 64;  // 0 .. 32*NUM_EPI_WARPS-1
+    bool ok = true;
+    if (C::B_NF4) {
+      const int64_t kblocks = p.w_k / 64;
+      // Row of the B tile this thread fills, and which weight block goes there.
+      const int n_local = C::B_MN ? (dt & 63) : dt;
+      const int slab = C::B_MN ? (dt >> 6) : 0;
+      const uint32_t row_off = static_cast<uint32_t>(slab) * 8192u + static_cast<uint32_t>(n_local) * 128u;
+      const uint32_t code_off = C::B_MN ? static_cast<uint32_t>(slab) * 2048u + static_cast<uint32_t>(n_local) * 32u
+                                        : static_cast<uint32_t>(dt) * 32u;
+      const uint32_t first_half = ((lane >> 2) & 1u) ? 16u : 0u;
+      const uint32_t sw = static_cast<uint32_t>(n_local & 7);
+      // Block index of step `it` for this thread, or -1 outside the weight.
+      auto block_of = [&](int it) -> int64_t {
+        int64_t gn, kb;
+        if (!C::B_MN) {
+          gn = static_cast<int64_t>(n_tile) * C::BN + dt;
+          kb = it;
+        } else {
+          gn = static_cast<int64_t>(it) * kBK + n_local;
+          kb = static_cast<int64_t>(n_tile) * (C::BN / 64) + slab;
+        }
+        return (gn < p.w_n && kb < kblocks) ? gn * kblocks + kb : -1;
+      };
+      // The absmax code and group constant of the next step are fetched one
+      // step ahead so their latency hides behind the current decode.
+      int64_t blk_nx = p.num_main > 0 ? block_of(0) : -1;
+      uint32_t q_nx = 0;
+      float S_nx = 0.f;
+      if (blk_nx >= 0) {
+        q_nx = __ldg(p.absmax_q + blk_nx);
+        S_nx = __ldg(p.group_scale + (blk_nx >> 8));
+      }
+      for (int it = 0; it < total; ++it) {
+        const int s = it % C::STAGES;
+        const uint32_t ph = static_cast<uint32_t>(it / C::STAGES) & 1u;
+        if (!mbar_wait_bounded(&full_a[s], ph, p.err, kErrTimeoutFullA)) { ok = false; break; }
+        if (it < p.num_main) {
+          const int64_t blk = blk_nx;
+          const uint32_t qv = q_nx;
+          const float S = S_nx;
+          if (it + 1 < p.num_main) {
+            blk_nx = block_of(it + 1);
+            if (blk_nx >= 0) {
+              q_nx = __ldg(p.absmax_q + blk_nx);
+              S_nx = __ldg(p.group_scale + (blk_nx >> 8));
+            }
+          }
+          const uint32_t a_s = base + static_cast<uint32_t>(s) * C::STAGE_BYTES;
+          const uint32_t b_s = a_s + C::A_BYTES;
+          const uint32_t c_s = b_s + C::B_BYTES;
+          Bf16Table tb;
+          uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = make_uint4(0u, 0u, 0u, 0u);
+          if (blk >= 0) {
+            const uint4 f = lds128(c_s + code_off + first_half);
+            const uint4 g2 = lds128(c_s + code_off + (16u - first_half));
+            lo = first_half ? g2 : f;
+            hi = first_half ? f : g2;
+            make_table(p.tab, absmax_dequant(qv, S), tb);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tb.lo[j] = tb.hi[j] = 0u;
+          }
+          const uint32_t words[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+          const uint32_t rowaddr = b_s + row_off;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t o[4];
+            decode8(words[c], tb, o);
+            sts128(rowaddr + ((static_cast<uint32_t>(c) ^ sw) << 4), o);
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full_b[s]);
+      }
+    }
+
+    // ------------------------------------------------------------ epilogue
+    if (ok) ok = mbar_wait_bounded(&acc_bar, 0u, p.err, kErrTimeoutAcc, 20000000000ull);
+    if (ok) {
+      tc_fence_after();
+      const int ew = warp - 2;
+      const int quad = warp & 3;
+      int h = 0, c_begin = 0, c_end = C::BN;
+      if (C::NUM_EPI_WARPS == 8) {
+        if (C::MSUB == 2) {
+          h = ew >> 2;
+        } else {
+          c_begin = (ew >> 2) * (C::BN / 2);
+          c_end = c_begin + C::BN / 2;
+        }
+      }
+      const int row_in_tile = h * 128 + quad * 32 + lane;
+      const int64_t grow = static_cast<int64_t>(m_tile) * C::BM + row_in_tile;
+      const bool row_ok = grow < p.out_rows;
+      for (int c0 = c_begin; c0 < c_end; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(h * C::BN + c0), v);
+        const int64_t gcol = static_cast<int64_t>(n_tile) * C::BN + c0;
+        if (!C::OUT_T) {
+          if (row_ok) {
+            uint16_t *dst = p.out + grow * p.out_ld + gcol;
+            if (gcol + 32 <= p.out_cols) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                uint4 w;
+                w.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]) * p.alpha, __uint_as_float(v[8 * j + 1]) * p.alpha);
+                w.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]) * p.alpha, __uint_as_float(v[8 * j + 3]) * p.alpha);
+                w.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]) * p.alpha, __uint_as_float(v[8 * j + 5]) * p.alpha);
+                w.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]) * p.alpha, __uint_as_float(v[8 * j + 7]) * p.alpha);
+                reinterpret_cast<uint4 *>(dst)[j] = w;
+              }
+            } else {
+              for (int j = 0; j < 32; ++j)
+                if (gcol + j < p.out_cols)
+                  dst[j] = static_cast<uint16_t>(pack_bf16x2(__uint_as_float(v[j]) * p.alpha, 0.f) & 0xFFFFu);
+            }
+          }
+        } else {
+          if (row_ok) {
+            for (int j = 0; j < 32; ++j)
+              if (gcol + j < p.out_cols)
+                p.out[(gcol + j) * p.out_ld + grow] =
+                    static_cast<uint16_t>(pack_bf16x2(__uint_as_float(v[j]) * p.alpha, 0.f) & 0xFFFFu);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS) : "memory");
+  }
+}
+
+// ---- host side ------------------------------------------------------------
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+// 2D map over a row-major [outer x inner] tensor with a row pitch in bytes.
+bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool map_bf16(CUtensorMap *m, const uint16_t *ptr, int64_t rows, int64_t cols, uint32_t box_cols, uint32_t box_rows) {
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, static_cast<uint64_t>(cols), static_cast<uint64_t>(rows),
+                  static_cast<uint64_t>(cols) * 2u, box_cols, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool map_codes(CUtensorMap *m, const uint8_t *ptr, int64_t rows, int64_t row_bytes, uint32_t box_bytes,
+               uint32_t box_rows) {
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, ptr, static_cast<uint64_t>(row_bytes),
+                  static_cast<uint64_t>(rows), static_cast<uint64_t>(row_bytes), box_bytes, box_rows,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+template <class C>
+cudaError_t launch(const TcParams &p, int grid_n, int grid_m, cudaStream_t stream) {
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !configured[dev]) {
+    e = cudaFuncSetAttribute(tc_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(C::SMEM_BYTES));
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) configured[dev] = true;
+  }
+  if (grid_n <= 0 || grid_m <= 0) return cudaSuccess;
+  tc_kernel<C><<<dim3(grid_n, grid_m, 1), C::NUM_THREADS, C::SMEM_BYTES, stream>>>(p);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+
+using CfgFwd2 = Cfg<256, 2, false, true, false, false>;
+using CfgFwd1 = Cfg<256, 1, false, true, false, false>;
+using CfgBwd2 = Cfg<256, 2, false, true, true, false>;
+using CfgBwd1 = Cfg<256, 1, false, true, true, false>;
+using CfgProjK = Cfg<64, 1, false, false, false, false>;
+using CfgProjMN = Cfg<64, 1, false, false, true, false>;
+using CfgTN = Cfg<64, 1, true, false, true, false>;
+using CfgTNT = Cfg<64, 1, true, false, true, true>;
+
+}  // namespace
+
+cudaError_t tc_fwd(const uint16_t *X, int64_t m, const WeightView &w, const uint16_t *T, const uint16_t *B,
+                   int32_t r, uint16_t *Y, cudaStream_t stream) {
+  TcParams p{};
+  const bool big = m > 128;
+  const uint32_t bm = big ? 256u : 128u;
+  const bool lora = T != nullptr && B != nullptr && r > 0;
+  if (!map_bf16(&p.tmA, X, m, w.k, 64, 128)) return cudaErrorInvalidValue;
+  if (!map_codes(&p.tmCodes, w.codes, w.n, w.k / 2, 32, 256)) return cudaErrorInvalidValue;
+  if (lora) {
+    if (!map_bf16(&p.tmA2, T, m, r, 64, 128)) return cudaErrorInvalidValue;
+    if (!map_bf16(&p.tmB2, B, w.n, r, 64, 256)) return cudaErrorInvalidValue;
+  }
+  p.absmax_q = w.absmax_q;
+  p.group_scale = w.group_scale;
+  p.out = Y;
+  p.err = device_error_word();
+  p.w_n = w.n;
+  p.w_k = w.k;
+  p.out_ld = w.n;
+  p.out_rows = static_cast<int>(m);
+  p.out_cols = static_cast<int>(w.n);
+  p.num_main = static_cast<int>(w.k / 64);
+  p.num_lora = lora ? cdiv(r, 64) : 0;
+  p.alpha = 1.0f;
+  p.tab = nf4_tables();
+  const int gn = cdiv(w.n, 256), gm = cdiv(m, bm);
+  return big ? launch<CfgFwd2>(p, gn, gm, stream) : launch<CfgFwd1>(p, gn, gm, stream);
+}
+
+cudaError_t tc_bwd_dx(const uint16_t *dY, int64_t m, const WeightView &w, const uint16_t *U, const uint16_t *A,
+                      int32_t r, uint16_t *dX, cudaStream_t stream) {
+  TcParams p{};
+  const bool big = m > 128;
+  const uint32_t bm = big ? 256u : 128u;
+  const bool lora = U != nullptr && A != nullptr && r > 0;
+  if (!map_bf16(&p.tmA, dY, m, w.n, 64, 128)) return cudaErrorInvalidValue;
+  if (!map_codes(&p.tmCodes, w.codes, w.n, w.k / 2, 32, 64)) return cudaErrorInvalidValue;
+  if (lora) {
+    if (!map_bf16(&p.tmA2, U, m, r, 64, 128)) return cudaErrorInvalidValue;
+    if (!map_bf16(&p.tmB2, A, r, w.k, 64, 64)) return cudaErrorInvalidValue;
+  }
+  p.absmax_q = w.absmax_q;
+  p.group_scale = w.group_scale;
+  p.out = dX;
+  p.err = device_error_word();
+  p.w_n = w.n;
+  p.w_k = w.k;
+  p.out_ld = w.k;
+  p.out_rows = static_cast<int>(m);
+  p.out_cols = static_cast<int>(w.k);
+  p.num_main = cdiv(w.n, 64);
+  p.num_lora = lora ? cdiv(r, 64) : 0;
+  p.alpha = 1.0f;
+  p.tab = nf4_tables();
+  const int gn = cdiv(w.k, 256), gm = cdiv(m, bm);
+  return big ? launch<CfgBwd2>(p, gn, gm, stream) : launch<CfgBwd1>(p, gn, gm, stream);
+}
+
+cudaError_t tc_proj_kmajor(const uint16_t *L, int64_t m, int64_t kc, const uint16_t *R, int32_t r, float scale,
+                           uint16_t *out, cudaStream_t stream) {
+  TcParams p{};
+  if (!map_bf16(&p.tmA, L, m, kc, 64, 128)) return cudaErrorInvalidValue;
+  if (!map_bf16(&p.tmB, R, r, kc, 64, 64)) return cudaErrorInvalidValue;
+  p.out = out;
+  p.err = device_error_word();
+  p.out_ld = r;
+  p.out_rows = static_cast<int>(m);
+  p.out_cols = r;
+  p.num_main = cdiv(kc, 64);
+  p.num_lora = 0;
+  p.alpha = scale;
+  return launch<CfgProjK>(p, cdiv(r, 64), cdiv(m, 128), stream);
+}
+
+cudaError_t tc_proj_mnmajor(const uint16_t *L, int64_t m, int64_t kc, const uint16_t *R, int32_t r, float scale,
+                            uint16_t *out, cudaStream_t stream) {
+  TcParams p{};
+  if (!map_bf16(&p.tmA, L, m, kc, 64, 128)) return cudaErrorInvalidValue;
+  if (!map_bf16(&p.tmB, R, kc, r, 64, 64)) return cudaErrorInvalidValue;
+  p.out = out;
+  p.err = device_error_word();
+  p.out_ld = r;
+  p.out_rows = static_cast<int>(m);
+  p.out_cols = r;
+  p.num_main = cdiv(kc, 64);
+  p.num_lora = 0;
+  p.alpha = scale;
+  return launch<CfgProjMN>(p, cdiv(r, 64), cdiv(m, 128), stream);
+}
+
+cudaError_t tc_tn_skinny(const uint16_t *Lt, int64_t mc, int64_t pdim, const uint16_t *R, int32_t r, uint16_t *out,
+                         bool transposed, cudaStream_t stream) {
+  TcParams p{};
+  if (!map_bf16(&p.tmA, Lt, mc, pdim, 64, 64)) return cudaErrorInvalidValue;
+  if (!map_bf16(&p.tmB, R, mc, r, 64, 64)) return cudaErrorInvalidValue;
+  p.out = out;
+  p.err = device_error_word();
+  p.out_ld = transposed ? pdim : r;
+  p.out_rows = static_cast<int>(pdim);
+  p.out_cols = r;
+  p.num_main = cdiv(mc, 64);
+  p.num_lora = 0;
+  p.alpha = 1.0f;
+  return transposed ? launch<CfgTNT>(p, cdiv(r, 64), cdiv(pdim, 128), stream)
+                    : launch<CfgTN>(p, cdiv(r, 64), cdiv(pdim, 128), stream);
+}
+
+}  // namespace qlora

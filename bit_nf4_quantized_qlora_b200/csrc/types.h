@@ -1,0 +1,26 @@
+// Plain types shared by host and device code of libqlora.
+#pragma once
+
+#include <cstdint>
+
+namespace qlora {
+
+// The fp32 codebook and the 15 decision midpoints, passed by value as a
+// kernel parameter (uniform across the grid).
+struct Nf4Tables {
+  float level[16];
+  float mid[15];
+  float pad_;
+};
+
+// Device-side error codes written to the caller-visible error word when a
+// bounded wait gives up (no kernel ever traps).
+enum : unsigned {
+  kErrTimeoutFullA = 1u << 0,
+  kErrTimeoutFullB = 1u << 1,
+  kErrTimeoutEmpty = 1u << 2,
+  kErrTimeoutAcc = 1u << 3,
+  kErrTimeoutDrain = 1u << 4,
+};
+
+}  // namespace qlora

@@ -1,0 +1,205 @@
+/*
+ * qlora.h -- C ABI of the NF4 + double-quantized QLoRA linear layer on B200.
+ *
+ * The layer (cited by web-page title and section):
+ *
+ *     Y = X . dequant(W)^T + s . (X . A^T) . B^T ,     s = alpha / r
+ *
+ *   - the frozen base weight W is stored in 4 bits and dequantized block by
+ *     block to bf16 for each matrix product ["QLoRA", Storage precision is not
+ *     calculation precision; "QLoRA and Quantized Training", The idea;
+ *     "A 65B fine-tune on the GPU you already have", figure 2];
+ *   - the 16 code levels sit at normal quantiles (NF4) ["QLoRA and Quantized
+ *     Training", The idea; "QLoRA Explained", 1. 4-bit NormalFloat];
+ *   - one absmax constant per block of 64 weights, and those constants are
+ *     themselves quantized to 8 bits in blocks of 256 with one fp32 constant
+ *     each ["A 65B fine-tune on the GPU you already have", figure 4;
+ *     "QLoRA > Summary"];
+ *   - only the low-rank adapters A, B (bf16) receive gradients; the input
+ *     gradient flows through the frozen dequantized weight ["QLoRA", Follow
+ *     one QLoRA training step; "QLoRA Explained", What is QLoRA?].
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers, allocated and owned by the
+ *     caller.  The library never allocates, frees or retains memory; scratch
+ *     space is a caller-provided workspace sized by qlora_workspace_bytes().
+ *   - Matrices are dense row-major.  bf16 tensors are passed as uint16_t bit
+ *     patterns (the layout of __nv_bfloat16).  W is [n x k] (out x in),
+ *     X [m x k], Y [m x n], A [r x k], B [n x r].
+ *   - Every tensor pointer must be 16-byte aligned.
+ *   - Shapes: n > 0, k > 0, k % 64 == 0; the linear operations also need
+ *     n % 8 == 0 (16-byte bf16 rows of Y and dY);
+ *     r % 16 == 0 with 0 <= r <= 256 (r == 0, or A == B == NULL, means no
+ *     adapter), m >= 0 (m == 0 is an empty batch: nothing is launched).
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream);
+ *     inputs must stay valid and outputs untouched until the stream reaches
+ *     the call.  All arguments are validated on the host before any launch:
+ *     a call that returns an error has launched nothing.  No kernel traps.
+ *   - Return value: QLORA_OK or one of the negative codes below.  After
+ *     QLORA_ERR_CUDA, qlora_last_cuda_error() returns the cudaError_t.
+ *   - Inputs must be finite (NaN/Inf weights are a documented precondition,
+ *     not checked on the device).
+ */
+#ifndef QLORA_H
+#define QLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; a cudaStream_t can be passed directly. */
+typedef struct CUstream_st *qlora_stream_t;
+
+enum qlora_status {
+  QLORA_OK = 0,
+  QLORA_ERR_NULL = -1,      /* a required pointer is NULL                  */
+  QLORA_ERR_SHAPE = -2,     /* a size breaks the shape rules above         */
+  QLORA_ERR_ALIGN = -3,     /* a pointer is not 16-byte aligned            */
+  QLORA_ERR_WORKSPACE = -4, /* workspace missing or smaller than required  */
+  QLORA_ERR_CUDA = -5,      /* a CUDA call failed (see last_cuda_error)    */
+  QLORA_ERR_DEVICE = -6     /* the current device is not sm_100            */
+};
+
+/* Quantized weight: three flat buffers plus the shape.
+ *   codes       uint8 [n*k/2]   NF4 codes, two per byte in row-major element
+ *                               order: byte j = (code[2j] << 4) | code[2j+1]
+ *   absmax_q    uint8 [n*k/64]  8-bit code of each block's absmax
+ *   group_scale fp32  [ceil(n*k/64/256)]  max absmax of each group of 256
+ *   block == 64 and group == 256 are the only supported values.
+ * Dequantization ["A 65B fine-tune on the GPU you already have", figure 4;
+ * "QLoRA", Storage precision is not calculation precision]:
+ *   c'  = fp32(float(absmax_q[b]) * fp32(group_scale[b/256] / 255))
+ *   W^  = bf16_rne(fp32(NF4[code] * c'))                                   */
+typedef struct {
+  const uint8_t *codes;
+  const uint8_t *absmax_q;
+  const float *group_scale;
+  int64_t n, k;
+  int32_t block;
+  int32_t group;
+} qlora_nf4_weight;
+
+/* Operation ids for qlora_workspace_bytes. */
+enum qlora_op { QLORA_OP_FWD = 0, QLORA_OP_BWD_DX = 1, QLORA_OP_LORA_BWD = 2 };
+
+/* Blockwise NF4 quantization with double-quantized absmax.
+ * ["QLoRA and Quantized Training", The idea and Worked example (blocks of 64,
+ *  one fp32 scale each, 0.5 byte per weight); "A 65B fine-tune on the GPU you
+ *  already have", figures 3 and 4 (NF4 levels; 8-bit constants in blocks of
+ *  256); "QLoRA > Summary" (scales quantized to 8-bit integers)]
+ *   W              in   fp32 [n x k]
+ *   codes          out  uint8 [n*k/2]
+ *   absmax_q       out  uint8 [n*k/64]
+ *   group_scale    out  fp32  [ceil(n*k/64/256)]
+ *   absmax_fp32    out  fp32  [n*k/64] block absmax before double
+ *                       quantization; may be NULL
+ * Per block b of 64 consecutive row-major weights: c_b = max|w|;
+ * code = #{i : fp32(w / c_b) > T_i} over the 15 fp32 midpoints T_i of the
+ * sorted NF4 levels (a value on a midpoint takes the lower code; c_b == 0
+ * gives code 7, the zero level).  Per group g of 256 blocks: S_g = max c_b,
+ * absmax_q = rint_even(fp32(fp32(c_b / S_g) * 255)) (0 when S_g == 0).     */
+int qlora_quantize_nf4_dq(const float *W, int64_t n, int64_t k,
+                          uint8_t *codes, uint8_t *absmax_q, float *group_scale,
+                          float *absmax_fp32, qlora_stream_t stream);
+
+/* Standalone dequantization to bf16 ["QLoRA", Storage precision is not
+ * calculation precision; "A 65B fine-tune on the GPU you already have",
+ * figure 2].
+ *   w       in   quantized weight [n x k]
+ *   W_bf16  out  bf16 [n x k], bit-exact W^ as defined at qlora_nf4_weight. */
+int qlora_dequant(const qlora_nf4_weight *w, uint16_t *W_bf16, qlora_stream_t stream);
+
+/* Forward: Y = bf16( X . W^T + T . B^T ),  T = bf16(s . X . A^T)
+ * ["QLoRA and Quantized Training", The idea (compute in bf16, each block
+ *  dequantized, used, discarded); "A 65B fine-tune on the GPU you already
+ *  have", figure 2; LoRA r and alpha from "QLoRA and Quantized Training",
+ *  In code]
+ *   X      in   bf16 [m x k]
+ *   w      in   quantized weight [n x k]
+ *   A, B   in   bf16 [r x k], [n x r]; NULL/NULL or r == 0: no adapter
+ *   scale  in   s = alpha / r
+ *   Y      out  bf16 [m x n]
+ *   ws     scratch, ws_bytes >= qlora_workspace_bytes(QLORA_OP_FWD, m, n, k, r);
+ *          contents on entry are ignored.
+ * Products accumulate in fp32.  m <= 16 runs a weight-streaming kernel; larger
+ * m runs the tcgen05 tensor-core kernel with dequantization in its main loop. */
+int qlora_linear_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w,
+                     const uint16_t *A, const uint16_t *B, int32_t r, float scale,
+                     uint16_t *Y, void *ws, size_t ws_bytes, qlora_stream_t stream);
+
+/* Input gradient: dX = bf16( dY . W^ + U . A ),  U = bf16(s . dY . B)
+ * ["QLoRA", Follow one QLoRA training step, step 4 (gradients flow into the
+ *  adapters, not the frozen base); "QLoRA Explained", What is QLoRA?
+ *  (backpropagates through a frozen, 4-bit quantized base model)]
+ *   dY     in   bf16 [m x n]
+ *   w      in   quantized weight [n x k]
+ *   A, B   in   bf16 [r x k], [n x r] (as in the forward)
+ *   dX     out  bf16 [m x k]
+ *   ws     scratch, ws_bytes >= qlora_workspace_bytes(QLORA_OP_BWD_DX, m, n, k, r) */
+int qlora_linear_bwd_dx(const uint16_t *dY, int64_t m, const qlora_nf4_weight *w,
+                        const uint16_t *A, const uint16_t *B, int32_t r, float scale,
+                        uint16_t *dX, void *ws, size_t ws_bytes, qlora_stream_t stream);
+
+/* Adapter gradients ["QLoRA and Quantized Training", The idea (the adapters
+ * hold the gradients and optimizer state); "QLoRA", Follow one QLoRA training
+ * step, step 4]:
+ *   dA = bf16( s . (dY . B)^T . X )      [r x k]
+ *   dB = bf16( dY^T . T ),  T = bf16(s . X . A^T)     [n x r]
+ *   X, dY  in   bf16 [m x k], [m x n]
+ *   A, B   in   bf16 [r x k], [n x r], r > 0
+ *   dA, dB out  bf16; overwritten (not accumulated)
+ *   ws     scratch, ws_bytes >= qlora_workspace_bytes(QLORA_OP_LORA_BWD, m, n, k, r)
+ * m == 0 writes zeros to dA and dB.                                        */
+int qlora_lora_bwd(const uint16_t *X, const uint16_t *dY, int64_t m, int64_t n, int64_t k,
+                   const uint16_t *A, const uint16_t *B, int32_t r, float scale,
+                   uint16_t *dA, uint16_t *dB, void *ws, size_t ws_bytes,
+                   qlora_stream_t stream);
+
+/* Workspace bytes an operation needs (0 if none); SIZE_MAX for an unknown op
+ * or invalid sizes.  A workspace may be reused across calls on one stream;
+ * two calls that may run concurrently need separate workspaces.             */
+size_t qlora_workspace_bytes(int op, int64_t m, int64_t n, int64_t k, int32_t r);
+
+/* cudaError_t of the last failing CUDA call on this host thread (0 if none). */
+int qlora_last_cuda_error(void);
+
+/* Device-side status: kernels never trap; a wait inside a kernel that gives
+ * up after its time limit sets a bit in a per-device error word instead and
+ * the kernel exits early (its outputs are then undefined).  This call
+ * synchronizes `stream`, writes the word to *flags (host memory; 0 = no
+ * error) and clears it.  QLORA_ERR_NULL if flags is NULL.                   */
+int qlora_poll_device_error(qlora_stream_t stream, unsigned *flags);
+
+/* Profiling hook.  While set, qlora_linear_fwd and qlora_linear_bwd_dx
+ * record `start` on their stream right before launching their main kernel
+ * (the fused tensor-core GEMM, or the weight-streaming kernel for small m)
+ * and `stop` right after it, so the caller can time that kernel alone with
+ * cudaEventElapsedTime.  Both are cudaEvent_t handles owned by the caller;
+ * the setting is per host thread; pass NULL, NULL to clear.  Returns
+ * QLORA_ERR_NULL if exactly one of the two is NULL.                         */
+int qlora_set_profile_events(void *start, void *stop);
+
+/* Number of CUDA kernels this library has launched in this process so far
+ * (all threads, all devices).  Lets a caller count the launches inside a
+ * timed region.                                                             */
+uint64_t qlora_launch_count(void);
+
+/* Static, human-readable name of a status code. */
+const char *qlora_status_string(int status);
+
+/* The library's own fp32 NF4 codebook, derived at load time from the normal
+ * quantile construction (16 ascending levels, index 7 == 0, 0 == -1,
+ * 15 == +1).  Host function; writes 16 floats to `levels` (host memory).   */
+void qlora_nf4_levels(float *levels);
+
+/* ABI version: (major << 16) | minor. */
+int qlora_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H */

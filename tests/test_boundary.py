@@ -1,0 +1,163 @@
+"""The C-ABI library: it loads, exports every symbol include/qlora.h declares,
+derives the same fp32 NF4 codebook as the oracle, and rejects bad arguments
+on the host before any launch.  No GPU is touched: every call here returns
+before the library's first CUDA call (fake device pointers are never
+dereferenced)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+from bit_nf4_quantized_qlora_b200 import binding as B
+from oracle import nf4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(HEADER_DIR):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(HEADER_DIR, fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(qlora_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return B.lib()
+
+
+def test_header_declares_the_five_entry_points():
+    names = _declared_functions()
+    for n in ("qlora_quantize_nf4_dq", "qlora_dequant", "qlora_linear_fwd", "qlora_linear_bwd_dx",
+              "qlora_lora_bwd", "qlora_workspace_bytes"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert len(names) >= 10
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in names:
+        assert n in exported, n
+        assert hasattr(lib, n)
+
+
+def test_library_codebook_equals_oracle_codebook(lib):
+    """The library derives its levels with its own inverse-normal routine; the
+    fp32 values must equal the oracle's bit for bit."""
+    got = np.array(B.qlora_nf4_levels(), dtype=np.float32)
+    assert np.array_equal(got.view(np.uint32), nf4.levels_f32().view(np.uint32))
+
+
+def test_version_and_status_strings(lib):
+    assert lib.qlora_version() >> 16 == 1
+    for st in (0, -1, -2, -3, -4, -5, -6):
+        assert lib.qlora_status_string(st)
+
+
+def test_workspace_bytes(lib):
+    f = B.qlora_workspace_bytes
+    assert f(B.QLORA_OP_FWD, 4096, 11008, 4096, 0) == 0
+    assert f(B.QLORA_OP_FWD, 4096, 11008, 4096, 64) == 4096 * 64 * 2
+    assert f(B.QLORA_OP_FWD, 3, 1024, 1024, 16) == 256          # rounded up to 256 B
+    assert f(B.QLORA_OP_BWD_DX, 16, 1024, 1024, 16) == 512
+    assert f(B.QLORA_OP_LORA_BWD, 16, 1024, 1024, 16) == 1024
+    assert f(99, 1, 1, 1, 1) == 2 ** 64 - 1
+    assert f(B.QLORA_OP_FWD, -1, 1, 1, 1) == 2 ** 64 - 1
+
+
+# ---- host-side validation (fake, aligned device addresses) -----------------
+
+P = 0x10000000          # a 16-byte aligned fake address, never dereferenced
+MIS = P + 8             # misaligned
+
+
+def _w(n=1024, k=1024, codes=P, q=P, s=P, block=64, group=256):
+    return B.NF4WeightC(codes, q, s, n, k, block, group)
+
+
+def _fwd(lib, X=P, m=16, w=None, A=P, Bm=P, r=16, Y=P, ws=P, ws_bytes=1 << 20):
+    w = w if w is not None else _w()
+    return lib.qlora_linear_fwd(X, m, ctypes.byref(w), A, Bm, r, 2.0, Y, ws, ws_bytes, None)
+
+
+def test_fwd_rejects_bad_arguments(lib):
+    assert _fwd(lib, X=None) == B.QLORA_ERR_NULL
+    assert _fwd(lib, Y=None) == B.QLORA_ERR_NULL
+    assert _fwd(lib, w=_w(codes=0)) == B.QLORA_ERR_NULL
+    assert _fwd(lib, w=_w(k=1000)) == B.QLORA_ERR_SHAPE           # k % 64
+    assert _fwd(lib, w=_w(n=1020)) == B.QLORA_ERR_SHAPE           # n % 8
+    assert _fwd(lib, w=_w(n=0)) == B.QLORA_ERR_SHAPE
+    assert _fwd(lib, w=_w(block=32)) == B.QLORA_ERR_SHAPE
+    assert _fwd(lib, w=_w(group=128)) == B.QLORA_ERR_SHAPE
+    assert _fwd(lib, r=12) == B.QLORA_ERR_SHAPE                    # r % 16
+    assert _fwd(lib, r=-16) == B.QLORA_ERR_SHAPE
+    assert _fwd(lib, m=-1) == B.QLORA_ERR_SHAPE
+    assert _fwd(lib, A=None) == B.QLORA_ERR_NULL                   # one adapter pointer
+    assert _fwd(lib, X=MIS) == B.QLORA_ERR_ALIGN
+    assert _fwd(lib, Y=MIS) == B.QLORA_ERR_ALIGN
+    assert _fwd(lib, A=MIS) == B.QLORA_ERR_ALIGN
+    assert _fwd(lib, w=_w(codes=MIS)) == B.QLORA_ERR_ALIGN
+    assert _fwd(lib, ws=None) == B.QLORA_ERR_WORKSPACE
+    assert _fwd(lib, ws_bytes=16 * 16 * 2 - 1) == B.QLORA_ERR_WORKSPACE
+    assert _fwd(lib, ws=MIS) == B.QLORA_ERR_ALIGN
+
+
+def test_fwd_empty_batch_is_a_no_op(lib):
+    assert _fwd(lib, m=0, X=None, Y=None, ws=None) == B.QLORA_OK
+
+
+def test_bwd_dx_rejects_bad_arguments(lib):
+    w = _w()
+    f = lambda **kw: lib.qlora_linear_bwd_dx(kw.get("dY", P), kw.get("m", 16), ctypes.byref(kw.get("w", w)),
+                                             kw.get("A", P), kw.get("B", P), kw.get("r", 16), 2.0,
+                                             kw.get("dX", P), kw.get("ws", P), kw.get("ws_bytes", 1 << 20), None)
+    assert f(dY=None) == B.QLORA_ERR_NULL
+    assert f(dX=MIS) == B.QLORA_ERR_ALIGN
+    assert f(w=_w(k=96)) == B.QLORA_ERR_SHAPE
+    assert f(ws_bytes=10) == B.QLORA_ERR_WORKSPACE
+    assert f(m=0, dY=None, dX=None) == B.QLORA_OK
+
+
+def test_lora_bwd_rejects_bad_arguments(lib):
+    f = lambda **kw: lib.qlora_lora_bwd(kw.get("X", P), kw.get("dY", P), kw.get("m", 16), kw.get("n", 1024),
+                                        kw.get("k", 1024), kw.get("A", P), kw.get("B", P), kw.get("r", 16), 2.0,
+                                        kw.get("dA", P), kw.get("dB", P), kw.get("ws", P),
+                                        kw.get("ws_bytes", 1 << 20), None)
+    assert f(A=None) == B.QLORA_ERR_NULL
+    assert f(dB=None) == B.QLORA_ERR_NULL
+    assert f(X=None) == B.QLORA_ERR_NULL
+    assert f(r=0) == B.QLORA_ERR_SHAPE
+    assert f(k=100) == B.QLORA_ERR_SHAPE
+    assert f(n=12) == B.QLORA_ERR_SHAPE
+    assert f(dA=MIS) == B.QLORA_ERR_ALIGN
+    assert f(ws=None) == B.QLORA_ERR_WORKSPACE
+    assert f(ws_bytes=1023) == B.QLORA_ERR_WORKSPACE
+
+
+def test_quantize_and_dequant_reject_bad_arguments(lib):
+    q = lambda **kw: lib.qlora_quantize_nf4_dq(kw.get("W", P), kw.get("n", 64), kw.get("k", 64), kw.get("c", P),
+                                               kw.get("q", P), kw.get("s", P), kw.get("a", None), None)
+    assert q(W=None) == B.QLORA_ERR_NULL
+    assert q(k=63) == B.QLORA_ERR_SHAPE
+    assert q(n=0) == B.QLORA_ERR_SHAPE
+    assert q(c=MIS) == B.QLORA_ERR_ALIGN
+    assert q(a=MIS) == B.QLORA_ERR_ALIGN
+    w = _w()
+    assert lib.qlora_dequant(ctypes.byref(w), None, None) == B.QLORA_ERR_NULL
+    assert lib.qlora_dequant(ctypes.byref(w), MIS, None) == B.QLORA_ERR_ALIGN
+    assert lib.qlora_dequant(None, P, None) == B.QLORA_ERR_NULL
+
+
+def test_poll_rejects_null(lib):
+    assert lib.qlora_poll_device_error(None, None) == B.QLORA_ERR_NULL
