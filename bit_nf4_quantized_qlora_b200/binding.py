@@ -73,6 +73,9 @@ _SIGNATURES = {
     "qlora_version": (ctypes.c_int, []),
     "qlora_set_profile_events": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_launch_count": (ctypes.c_uint64, []),
+    "qlora_linear_fwd_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(NF4WeightC),
+                                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_float,
+                                                ctypes.c_void_p, ctypes.c_void_p]),
 }
 
 
@@ -259,3 +262,21 @@ def qlora_lora_bwd(X: torch.Tensor, dY: torch.Tensor, A: torch.Tensor, B: torch.
            lib().qlora_lora_bwd(X.data_ptr(), dY.data_ptr(), m, n, k, A.data_ptr(), B.data_ptr(), r, float(scale),
                                 dA.data_ptr(), dB.data_ptr(), _ptr(ws), ws_bytes, _stream(stream)))
     return dA, dB
+
+
+def qlora_linear_fwd_noalloc(X: torch.Tensor, w: NF4Weight, A: Optional[torch.Tensor] = None,
+                             B: Optional[torch.Tensor] = None, r: int = 0, scale: float = 0.0,
+                             out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Forward without a workspace: the library's built-in device scratch
+    (QLORA_NOALLOC_SCRATCH_BYTES) holds T.  For callers that cannot allocate;
+    `out` must then be passed in."""
+    A, B, r = _lora_args(A, B, r)
+    _need_cuda(X, A, B, out)
+    m = X.shape[0]
+    if out is None:
+        out = torch.empty(m, w.n, dtype=torch.bfloat16, device=X.device)
+    ws_c = w.c_struct()
+    _check("qlora_linear_fwd_noalloc",
+           lib().qlora_linear_fwd_noalloc(X.data_ptr(), m, ctypes.byref(ws_c), _ptr(A), _ptr(B), r, float(scale),
+                                          out.data_ptr(), _stream(stream)))
+    return out

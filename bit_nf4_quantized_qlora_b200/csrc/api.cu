@@ -75,6 +75,8 @@ WeightView view(const qlora_nf4_weight *w) {
 
 }  // namespace
 
+int status_from_cuda(cudaError_t e) { return cuda_status(e); }
+
 void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
 unsigned *device_error_word() {

@@ -18,6 +18,10 @@ unsigned *device_error_word();
 // Process-wide count of kernel launches (see qlora_launch_count).
 void count_launches(int n);
 
+// QLORA_OK for cudaSuccess; otherwise records the error for
+// qlora_last_cuda_error() and returns QLORA_ERR_CUDA.
+int status_from_cuda(cudaError_t e);
+
 // --- launchers (all asynchronous on `stream`; return cudaError_t) --------
 
 cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q,

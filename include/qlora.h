@@ -158,6 +158,30 @@ int qlora_lora_bwd(const uint16_t *X, const uint16_t *dY, int64_t m, int64_t n, 
                    uint16_t *dA, uint16_t *dB, void *ws, size_t ws_bytes,
                    qlora_stream_t stream);
 
+/* Forward with no caller workspace, for callers that cannot allocate device
+ * memory: code whose host owns every device allocation (an engine plugin), a
+ * deployment that forbids allocation on its serving path, or a C caller with
+ * no device allocator.  The pages have no counterpart: this is a convenience
+ * of this library around qlora_linear_fwd.
+ *   Same arguments, semantics and results as qlora_linear_fwd, minus `ws`.
+ *   The rank-r scratch T lives in a fixed device array of
+ *   QLORA_NOALLOC_SCRATCH_BYTES inside the library; every device that loads
+ *   the library holds it until the process exits.  Calls whose scratch
+ *   (m*r*2 bytes rounded up to 256) exceeds it return QLORA_ERR_WORKSPACE and
+ *   launch nothing.  The call allocates nothing: no cudaMalloc, no cudaFree,
+ *   no allocating library routine.
+ *   The first call with an adapter on a device looks up the array's device
+ *   address (cudaGetSymbolAddress) with that device current; make that first
+ *   call before any stream capture.
+ *   All calls on a device share the array and it keeps the last call's
+ *   contents; T is fully written before it is read, so nothing in it needs to
+ *   start at zero.  Calls that may run at the same time on one device (other
+ *   streams, other host threads) race on the array: serialize them.        */
+#define QLORA_NOALLOC_SCRATCH_BYTES (1u << 20)
+int qlora_linear_fwd_noalloc(const uint16_t *X, int64_t m, const qlora_nf4_weight *w,
+                             const uint16_t *A, const uint16_t *B, int32_t r, float scale,
+                             uint16_t *Y, qlora_stream_t stream);
+
 /* Workspace bytes an operation needs (0 if none); SIZE_MAX for an unknown op
  * or invalid sizes.  A workspace may be reused across calls on one stream;
  * two calls that may run concurrently need separate workspaces.             */
