@@ -131,7 +131,7 @@ class ClockSampler:
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device_index: int, interval_s: float = 0.01):
+    def __init__(self, device_index: int, interval_s: float = 0.002):
         self.idx = device_index
         self.dt = interval_s
         self.samples = []
@@ -316,7 +316,7 @@ def _cpu_baseline(rank: int, world: int):
     if rank != 0 or world != 1:
         return None
     try:
-        return reference_step_sample(rows=48, repeat=1)
+        return reference_step_sample(rows=4096, out_rows_frac=1.0)
     except Exception as e:  # the oracle is a reported baseline only
         return {"value": None, "unit": UNIT, "kind": "oracle", "error": str(e)}
 
@@ -477,61 +477,53 @@ def _cpu_cores() -> int:
 _REF_CACHE = {}
 
 
-def _ref_prepare(rows: int):
-    """Untimed set-up of the oracle sample: per projection the fp32 weight,
-    `rows` token rows of X and dY, and A, B as exact fp64 values."""
-    if rows in _REF_CACHE:
-        return _REF_CACHE[rows]
+def _ref_prepare(rows: int, out_rows_frac: float):
+    """Untimed input generation for the oracle sample: per projection the
+    first `rows` token rows of X and dY, the first C = out_rows_frac * n weight
+    rows (C*k a whole number of 256-block groups), and A, B."""
+    key = (rows, out_rows_frac)
+    if key in _REF_CACHE:
+        return _REF_CACHE[key]
     import numpy as np
     import torch
     from bit_nf4_quantized_qlora_b200 import workloads as WL
     items = []
     for p in PROJECTIONS:
         c = WL.mlp_7b(p)
-        W = c.W().reshape(-1).numpy()
+        unit = 16384 // __import__("math").gcd(16384, c.k)        # rows per whole group boundary
+        C = max(unit, int(c.n * out_rows_frac) // unit * unit)
+        W = c.W()[:C].reshape(-1).numpy().copy()
         X = c.X()[:rows].to(torch.float32).numpy().astype(np.float64)
-        dY = c.dY()[:rows].to(torch.float32).numpy().astype(np.float64)
+        dY = c.dY()[:rows, :C].to(torch.float32).numpy().astype(np.float64)
         A = c.A().to(torch.float32).numpy().astype(np.float64)
-        Bm = c.B().to(torch.float32).numpy().astype(np.float64)
-        items.append((c, W, X, dY, A, Bm))
-    _REF_CACHE[rows] = items
+        Bm = c.B()[:C].to(torch.float32).numpy().astype(np.float64)
+        items.append((c, C, W, X, dY, A, Bm))
+    _REF_CACHE[key] = items
     return items
 
 
-def reference_step_sample(rows: int = 8, repeat: int = 1, quant_groups: int = 64) -> dict:
-    """One bounded sample of the step through the oracle: for each projection,
-    quantize + dequantize `quant_groups` groups of 256 blocks of W, dequantize
-    the rest of W once, then fwd, bwd_dx and the adapter gradients for `rows`
-    token rows.  Returns TFLOP/s of the sampled linear algebra."""
-    import numpy as np
+def reference_step_sample(rows: int = 8, out_rows_frac: float = 1.0 / 64) -> dict:
+    """One bounded sample of the step through the oracle: for each projection
+    the sub-problem of `rows` tokens and C of its n output rows -- quantize and
+    dequantize those C weight rows, then fwd, bwd_dx and the adapter
+    gradients -- all timed.  Returns TFLOP/s of the sampled linear algebra."""
     from oracle import linear, quant
-    items = _ref_prepare(rows)
+    items = _ref_prepare(rows, out_rows_frac)
     flops = 0
-    t_total = 0.0
-    for _ in range(repeat):
-        for c, W, X, dY, A, Bm in items:
-            t = time.perf_counter()
-            sample = W[:quant_groups * 16384]
-            p, q, S, _ = quant.quantize_nf4_dq(sample)
-            quant.dequant_bf16_values(p, q, S)
-            t_q = time.perf_counter() - t
-            key = ("what", c.name)
-            if key not in _REF_CACHE:
-                pw, qw, sw, _ = quant.quantize_nf4_dq(W)
-                _REF_CACHE[key] = quant.dequant_bf16_values(pw, qw, sw).reshape(c.n, c.k)
-            W_hat = _REF_CACHE[key]
-            t = time.perf_counter()
-            linear.fwd(X, W_hat, A, Bm, c.scale)
-            linear.bwd_dx(dY, W_hat, A, Bm, c.scale)
-            linear.lora_grads(X, dY, A, Bm, c.scale)
-            t_total += time.perf_counter() - t + t_q
-            flops += linear_flops(rows, c.n, c.k, c.r)["total"]
-    value = flops / t_total / 1e12
-    return {"value": value, "unit": UNIT, "cores": _cpu_cores(), "kind": "oracle",
-            "sample": f"per projection (gate, up, down): oracle quantize+dequantize of {quant_groups} groups "
-                      f"({quant_groups * 16384} weights) and fwd + bwd_dx + LoRA grads in fp64 for {rows} of the "
-                      f"4096 token rows (W^ dequantized once, untimed)",
-            "seconds": round(t_total, 3)}
+    t0 = time.perf_counter()
+    for c, C, W, X, dY, A, Bm in items:
+        packed, q, S, _ = quant.quantize_nf4_dq(W)
+        W_hat = quant.dequant_bf16_values(packed, q, S).reshape(C, c.k)
+        linear.fwd(X, W_hat, A, Bm, c.scale)
+        linear.bwd_dx(dY, W_hat, A, Bm, c.scale)
+        linear.lora_grads(X, dY, A, Bm, c.scale)
+        flops += linear_flops(rows, C, c.k, c.r)["total"]
+    el = time.perf_counter() - t0
+    return {"value": flops / el / 1e12, "unit": UNIT, "cores": _cpu_cores(), "kind": "oracle",
+            "sample": f"per projection (gate, up, down): {rows} of the 4096 token rows x about "
+                      f"{out_rows_frac:.4g} of the output rows -- oracle quantize + dequantize of those weight "
+                      f"rows, fwd, bwd_dx and LoRA grads in fp64 (NumPy)",
+            "seconds": round(el, 3)}
 
 
 def run_reference(args):
@@ -539,12 +531,12 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return                                          # only rank 0 runs the oracle
-    rows = 8
-    _ref_prepare(rows)
+    rows, frac = 64, 1.0 / 64
+    _ref_prepare(rows, frac)
     for _ in range(args.warmup):
-        reference_step_sample(rows=rows)
+        reference_step_sample(rows=rows, out_rows_frac=frac)
     t = time.perf_counter()
-    vals = [reference_step_sample(rows=rows) for _ in range(args.steps)]
+    vals = [reference_step_sample(rows=rows, out_rows_frac=frac) for _ in range(args.steps)]
     el = time.perf_counter() - t
     value = sum(v["value"] for v in vals) / len(vals)
     sample = vals[0]

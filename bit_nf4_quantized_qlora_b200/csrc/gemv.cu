@@ -2,47 +2,56 @@
 //
 // At decode-sized M the layer is bound by reading the packed weights from HBM
 // ("QLoRA and Quantized Training", The idea: dequantize each block, multiply,
-// discard).  Each warp owns 16 weight rows and walks K in chunks of 256 (four
-// NF4 blocks per row); lane (g = lane/4, q = lane%4) streams the 32 bytes of
-// block q of rows g and g+8 with 16-byte loads, expands them to exact bf16 W^
-// in registers (per-block table, common.cuh) and feeds m16n8k16 tensor-core
-// MMAs whose A operand is X.  The MMA's k order inside a step is permuted to
-// match what each lane holds, and X is read with the same permutation.
+// discard), so the kernel is a streaming pipeline whose decode costs about one
+// byte permute and one shared-memory load per two weights:
 //
-// A CTA is 8 warps = 2 row groups x 4 K parts (32 rows).  A thread-block
-// cluster of 1..8 CTAs splits K further; partial sums meet in shared memory
-// and are reduced across the cluster through distributed shared memory, after
-// which the adapter term T . B^T is added and Y is written once in bf16.
+//   * one producer warp streams 16 KB tiles of packed codes (128 weight rows x
+//     4 NF4 blocks, 128-byte swizzled) into a shared-memory ring with TMA;
+//   * a 64 KB shared table maps every code byte (two weights) to the bf16 pair
+//     {NF4[hi nibble], NF4[lo nibble]}, with 32 lane-private copies 256 bytes
+//     apart so 32 lookups always hit 32 banks;
+//   * eight consumer warps (16 rows each) feed the pairs as the A operand of
+//     m16n8k16 tensor-core MMAs with X as the B operand; the four MMAs of an
+//     NF4 block accumulate into a fresh tile that is scaled by the block's
+//     reconstructed absmax c' = q * fp32(S/255) and added to the running sum;
+//   * a cluster of CTAs splits K; partial tiles are reduced through
+//     distributed shared memory and the adapter term T . B^T is added before
+//     Y is written once in bf16.  T comes from the preceding projection
+//     kernel, which this kernel overlaps (programmatic dependent launch) and
+//     waits for only before its epilogue.
+#include <cuda.h>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace qlora {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kNT = 2;                         // n8 tiles per warp
-constexpr int kRowsPerWarp = 8 * kNT;          // 16
-constexpr int kKParts = 4;
-constexpr int kRowGroups = (kThreads / 32) / kKParts;  // 2
-constexpr int kRows = kRowGroups * kRowsPerWarp;       // 32 rows per CTA
+constexpr int kConsumers = 8;
+constexpr int kThreads = 32 * (kConsumers + 1);       // + one producer warp
+constexpr int kRows = 16 * kConsumers;                 // 128 weight rows per CTA
+constexpr int kStageBlocks = 4;                        // NF4 blocks of K per stage
+constexpr uint32_t kStageBytes = kRows * kStageBlocks * 32u;   // 16 KB
+constexpr int kStages = 2;                             // x 2 CTAs per SM
 constexpr int kMaxM = 16;
+constexpr uint32_t kLutBytes = 256u * 256u;            // 256 entries x 256-byte stride
+constexpr uint32_t kSmemBytes = kLutBytes + 1024u + kStages * kStageBytes + kMaxM * kRows * 4u;
 
-struct GemvParams {
+struct __align__(64) GemvParams {
+  CUtensorMap tmCodes;          // codes as [n rows x k/2 bytes], box {128, 128}, 128B swizzle
   const uint16_t *X;
-  const uint8_t *codes;
   const uint8_t *absmax_q;
   const float *group_scale;
   const uint16_t *T;
   const uint16_t *B;
   uint16_t *Y;
+  unsigned *err;
   int64_t n, k;
   int m, r;
-  int nchunks;
   Nf4Tables tab;
 };
 
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                               uint32_t b1) {
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
@@ -63,109 +72,276 @@ __device__ __forceinline__ uint32_t cluster_size() {
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ float ld_dsmem_f32(const float *local, uint32_t rank) {
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t rank) {
   uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
   return v;
 }
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint64_t *bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
 
-__global__ void __launch_bounds__(kThreads) gemv_fwd_kernel(const __grid_constant__ GemvParams p) {
-  __shared__ float red[kKParts][kMaxM][kRows];
+// LUT offset of byte j (0..3) of `word` for this lane: (byte << 8) | lane*4.
+template <int J>
+__device__ __forceinline__ uint32_t lut_off(uint32_t word, uint32_t lane4) {
+  return prmt(word, lane4, 0x5504u | (J << 4));
+}
+
+// One NF4 block (4 MMA k-steps) of this lane's two rows: returns the block's
+// raw products (before its absmax scale) in bacc.
+template <int TOK_TILES>
+__device__ __forceinline__ void block_mma(float (&bacc)[TOK_TILES][4], uint2 c0, uint2 c1, const uint4 (&xa)[TOK_TILES],
+                                          const uint4 (&xb)[TOK_TILES], const uint8_t *lut, uint32_t lane4) {
+#pragma unroll
+  for (int t = 0; t < TOK_TILES; ++t) bacc[t][0] = bacc[t][1] = bacc[t][2] = bacc[t][3] = 0.f;
+#pragma unroll
+  for (int ss = 0; ss < 4; ++ss) {
+    const uint32_t w0 = ss < 2 ? c0.x : c0.y;
+    const uint32_t w1 = ss < 2 ? c1.x : c1.y;
+    uint32_t a[4];
+    if ((ss & 1) == 0) {
+      a[0] = *reinterpret_cast<const uint32_t *>(lut + lut_off<0>(w0, lane4));
+      a[1] = *reinterpret_cast<const uint32_t *>(lut + lut_off<0>(w1, lane4));
+      a[2] = *reinterpret_cast<const uint32_t *>(lut + lut_off<1>(w0, lane4));
+      a[3] = *reinterpret_cast<const uint32_t *>(lut + lut_off<1>(w1, lane4));
+    } else {
+      a[0] = *reinterpret_cast<const uint32_t *>(lut + lut_off<2>(w0, lane4));
+      a[1] = *reinterpret_cast<const uint32_t *>(lut + lut_off<2>(w1, lane4));
+      a[2] = *reinterpret_cast<const uint32_t *>(lut + lut_off<3>(w0, lane4));
+      a[3] = *reinterpret_cast<const uint32_t *>(lut + lut_off<3>(w1, lane4));
+    }
+#pragma unroll
+    for (int t = 0; t < TOK_TILES; ++t) {
+      const uint4 &xv = ss < 2 ? xa[t] : xb[t];
+      mma_16816(bacc[t], a, (ss & 1) ? xv.z : xv.x, (ss & 1) ? xv.w : xv.y);
+    }
+  }
+}
+
+// Absmax code byte j of a word -> float (exact for 0..255).
+template <int J>
+__device__ __forceinline__ float qbyte(uint32_t w) {
+  return __uint_as_float(prmt(w, 0x4B000000u, 0x7650u | J)) - 8388608.0f;
+}
+
+template <int TOK_TILES>
+__global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_constant__ GemvParams p) {
+  extern __shared__ __align__(16) uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t full_bar[kStages];
+  __shared__ __align__(8) uint64_t empty_bar[kStages];
+
+  // The byte-pair table sits at the start of dynamic shared memory (a
+  // link-time constant address); the TMA ring is 1024-aligned after it.
+  const uint8_t *lut = dsmem;
+  const uint32_t ring = (smem_u32(dsmem) + kLutBytes + 1023u) & ~1023u;
+  const uint32_t red_addr = ring + kStages * kStageBytes;
+  float *red = reinterpret_cast<float *>(dsmem + (red_addr - smem_u32(dsmem)));
 
   const uint32_t crank = cluster_rank();
   const uint32_t csize = cluster_size();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int g = lane >> 2, q = lane & 3;
-  const int rg = warp / kKParts, kp = warp % kKParts;
   const int64_t n_cta = static_cast<int64_t>(blockIdx.x) * kRows;
-  const int64_t kblocks = p.k / 64;
-  const int c_lo = static_cast<int>((static_cast<int64_t>(p.nchunks) * crank) / csize);
-  const int c_hi = static_cast<int>((static_cast<int64_t>(p.nchunks) * (crank + 1)) / csize);
+  const int kblocks = static_cast<int>(p.k / 64);
+  // This CTA's share of K in whole stages of 4 blocks (the last may be ragged).
+  const int nst_all = (kblocks + kStageBlocks - 1) / kStageBlocks;
+  const int st_lo = static_cast<int>((static_cast<int64_t>(nst_all) * crank) / csize);
+  const int st_hi = static_cast<int>((static_cast<int64_t>(nst_all) * (crank + 1)) / csize);
+  const int nst = st_hi - st_lo;
+  const int kb_lo = st_lo * kStageBlocks;
 
-  float acc[kNT][4];
-#pragma unroll
-  for (int t = 0; t < kNT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-
-  const bool row_lo_x = g < p.m;
-  const bool row_hi_x = g + 8 < p.m;
-
-#pragma unroll 1
-  for (int c = c_lo + kp; c < c_hi; c += kKParts) {
-    const int64_t kb = static_cast<int64_t>(c) * 4 + q;
-    const bool kvalid = kb < kblocks;
-    uint4 cw[kNT][2];
-    Bf16Table tb[kNT];
-#pragma unroll
-    for (int t = 0; t < kNT; ++t) {
-      const int64_t row = n_cta + rg * kRowsPerWarp + 8 * t + g;
-      if (kvalid && row < p.n) {
-        const int64_t blk = row * kblocks + kb;
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.codes + blk * 32);
-        cw[t][0] = __ldcs(src);
-        cw[t][1] = __ldcs(src + 1);
-        const uint32_t qv = __ldg(p.absmax_q + blk);
-        const float S = __ldg(p.group_scale + (blk >> 8));
-        make_table(p.tab, absmax_dequant(qv, S), tb[t]);
-      } else {
-        cw[t][0] = cw[t][1] = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) tb[t].lo[j] = tb[t].hi[j] = 0u;
-      }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kConsumers);
     }
-    const uint16_t *xg = p.X + static_cast<int64_t>(g) * p.k + kb * 64;
-    const uint16_t *x8 = p.X + static_cast<int64_t>(g + 8) * p.k + kb * 64;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      uint32_t P[kNT][4];
-#pragma unroll
-      for (int t = 0; t < kNT; ++t) {
-        const uint4 &v = cw[t][w >> 2];
-        const uint32_t word = (w & 3) == 0 ? v.x : (w & 3) == 1 ? v.y : (w & 3) == 2 ? v.z : v.w;
-        decode8(word, tb[t], P[t]);
-      }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int ss = 2 * w + h;
-        uint2 xa = make_uint2(0u, 0u), xb = make_uint2(0u, 0u);
-        if (kvalid && row_lo_x) xa = __ldg(reinterpret_cast<const uint2 *>(xg + 4 * ss));
-        if (kvalid && row_hi_x) xb = __ldg(reinterpret_cast<const uint2 *>(x8 + 4 * ss));
-        const uint32_t a[4] = {xa.x, xb.x, xa.y, xb.y};
-#pragma unroll
-        for (int t = 0; t < kNT; ++t) mma_bf16_16816(acc[t], a, P[t][2 * h], P[t][2 * h + 1]);
-      }
-    }
+    fence_mbar_init();
   }
-
-  // Partial sums of this warp: D[m][n] with m = g, g+8 and n = 2q, 2q+1.
-#pragma unroll
-  for (int t = 0; t < kNT; ++t) {
-    const int nl = rg * kRowsPerWarp + 8 * t + 2 * q;
-    red[kp][g][nl] = acc[t][0];
-    red[kp][g][nl + 1] = acc[t][1];
-    red[kp][g + 8][nl] = acc[t][2];
-    red[kp][g + 8][nl + 1] = acc[t][3];
+  {
+    // Entry b (256 bytes): 32 copies of the pair, written 4 copies per store.
+    uint4 *lw = reinterpret_cast<uint4 *>(dsmem);
+    for (int i = threadIdx.x; i < 256 * 8; i += kThreads) {
+      const int b = i >> 3;
+      const uint32_t v = pack_bf16x2(p.tab.level[b >> 4], p.tab.level[b & 15]);
+      lw[b * 16 + (i & 7)] = make_uint4(v, v, v, v);
+    }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < kMaxM * kRows; i += kThreads) {
-    float s = 0.f;
+
+  if (warp == kConsumers) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int st = 0; st < nst; ++st) {
+        const int s = st % kStages;
+        const uint32_t ph = static_cast<uint32_t>(st / kStages) & 1u;
+        if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, p.err, kErrTimeoutEmpty)) break;
+        mbar_arrive_expect_tx(&full_bar[s], kStageBytes);
+        tma_load_2d(ring + s * kStageBytes, &p.tmCodes, &full_bar[s], (kb_lo + st * kStageBlocks) * 32,
+                    static_cast<int>(n_cta));
+        ++issued;
+      }
+      for (int st = issued - kStages < 0 ? 0 : issued - kStages; st < issued; ++st)
+        mbar_wait_bounded(&full_bar[st % kStages], static_cast<uint32_t>(st / kStages) & 1u, p.err,
+                          kErrTimeoutDrain);
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const int g = lane >> 2, q = lane & 3;
+    const int lr0 = warp * 16 + g, lr1 = lr0 + 8;          // rows of the tile (rows past n are
+    const int64_t gr0 = n_cta + lr0 < p.n ? n_cta + lr0 : p.n - 1;   // computed but never stored)
+    const int64_t gr1 = n_cta + lr1 < p.n ? n_cta + lr1 : p.n - 1;
+    const int64_t b0 = gr0 * kblocks, b1 = gr1 * kblocks;
+    const uint8_t *q0p = p.absmax_q + b0 + kb_lo;
+    const uint8_t *q1p = p.absmax_q + b1 + kb_lo;
+    // Word loads of 4 absmax codes need 4-aligned block indices.
+    const bool qwords = (kblocks & 3) == 0;
+    const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
+    // Swizzled offsets (inside a stage tile) of this lane's 8 bytes of block b.
+    uint32_t off0[kStageBlocks], off1[kStageBlocks];
 #pragma unroll
-    for (int j = 0; j < kKParts; ++j) s += (&red[j][0][0])[i];
-    (&red[0][0][0])[i] = s;
+    for (int b = 0; b < kStageBlocks; ++b) {
+      const uint32_t chunk = ((2u * b + (q >> 1)) ^ static_cast<uint32_t>(g)) << 4;
+      off0[b] = static_cast<uint32_t>(lr0) * 128u + chunk + 8u * (q & 1);
+      off1[b] = static_cast<uint32_t>(lr1) * 128u + chunk + 8u * (q & 1);
+    }
+
+    // t = fp32(S / 255) of each row's current group and the block where the
+    // next group starts.
+    float t0 = 0.f, t1 = 0.f;
+    int next0 = kb_lo, next1 = kb_lo;
+
+    float acc[TOK_TILES][4];
+#pragma unroll
+    for (int t = 0; t < TOK_TILES; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+
+    const uint4 *xp[TOK_TILES];
+    bool xok[TOK_TILES];
+#pragma unroll
+    for (int t = 0; t < TOK_TILES; ++t) {
+      const int tok = g + 8 * t;
+      xok[t] = tok < p.m;
+      xp[t] = reinterpret_cast<const uint4 *>(p.X + static_cast<int64_t>(xok[t] ? tok : 0) * p.k +
+                                              static_cast<int64_t>(kb_lo) * 64 + 16 * q);
+    }
+
+    bool ok = true;
+    for (int st = 0; st < nst && ok; ++st) {
+      const int s = st % kStages;
+      const uint32_t ph = static_cast<uint32_t>(st / kStages) & 1u;
+      const int kb_st = kb_lo + st * kStageBlocks;
+      const bool full = kb_st + kStageBlocks <= kblocks;
+      // Absmax codes and X of this stage, issued before the wait.
+      float qf0[kStageBlocks], qf1[kStageBlocks];
+      if (full && qwords) {
+        const uint32_t w0 = __ldg(reinterpret_cast<const uint32_t *>(q0p + st * kStageBlocks));
+        const uint32_t w1 = __ldg(reinterpret_cast<const uint32_t *>(q1p + st * kStageBlocks));
+        qf0[0] = qbyte<0>(w0); qf0[1] = qbyte<1>(w0); qf0[2] = qbyte<2>(w0); qf0[3] = qbyte<3>(w0);
+        qf1[0] = qbyte<0>(w1); qf1[1] = qbyte<1>(w1); qf1[2] = qbyte<2>(w1); qf1[3] = qbyte<3>(w1);
+      } else {
+#pragma unroll
+        for (int b = 0; b < kStageBlocks; ++b) {
+          const bool v = kb_st + b < kblocks;
+          qf0[b] = v ? static_cast<float>(__ldg(q0p + st * kStageBlocks + b)) : 0.f;
+          qf1[b] = v ? static_cast<float>(__ldg(q1p + st * kStageBlocks + b)) : 0.f;
+        }
+      }
+      uint4 xa[kStageBlocks][TOK_TILES], xb[kStageBlocks][TOK_TILES];
+#pragma unroll
+      for (int b = 0; b < kStageBlocks; ++b) {
+#pragma unroll
+        for (int t = 0; t < TOK_TILES; ++t) {
+          xa[b][t] = make_uint4(0u, 0u, 0u, 0u);
+          xb[b][t] = make_uint4(0u, 0u, 0u, 0u);
+          if (xok[t] && (full || kb_st + b < kblocks)) {
+            xa[b][t] = __ldg(xp[t] + (st * kStageBlocks + b) * 8);
+            xb[b][t] = __ldg(xp[t] + (st * kStageBlocks + b) * 8 + 1);
+          }
+        }
+      }
+      // Group constants: with 4-aligned blocks a group boundary falls on a
+      // stage start; otherwise the slow path below takes it block by block.
+      if (kb_st >= next0) {
+        t0 = __fdiv_rn(__ldg(p.group_scale + ((b0 + kb_st) >> 8)), 255.0f);
+        next0 = kb_st + 256 - static_cast<int>((b0 + kb_st) & 255);
+      }
+      if (kb_st >= next1) {
+        t1 = __fdiv_rn(__ldg(p.group_scale + ((b1 + kb_st) >> 8)), 255.0f);
+        next1 = kb_st + 256 - static_cast<int>((b1 + kb_st) & 255);
+      }
+      ok = mbar_wait_bounded(&full_bar[s], ph, p.err, kErrTimeoutFullA);
+      if (!ok) break;
+      const uint32_t tile = ring + s * kStageBytes;
+      const bool fast = full && next0 >= kb_st + kStageBlocks && next1 >= kb_st + kStageBlocks;
+#pragma unroll
+      for (int b = 0; b < kStageBlocks; ++b) {
+        const uint2 c0 = lds64(tile + off0[b]);
+        const uint2 c1 = lds64(tile + off1[b]);
+        float bacc[TOK_TILES][4];
+        block_mma<TOK_TILES>(bacc, c0, c1, xa[b], xb[b], lut, lane4);
+        if (!fast) {
+          const int kb = kb_st + b;
+          if (kb == next0 && kb < kblocks) {
+            t0 = __fdiv_rn(__ldg(p.group_scale + ((b0 + kb) >> 8)), 255.0f);
+            next0 += 256;
+          }
+          if (kb == next1 && kb < kblocks) {
+            t1 = __fdiv_rn(__ldg(p.group_scale + ((b1 + kb) >> 8)), 255.0f);
+            next1 += 256;
+          }
+        }
+        // Blocks past K have q = 0 and add nothing.
+        const float s0 = __fmul_rn(qf0[b], t0);
+        const float s1 = __fmul_rn(qf1[b], t1);
+#pragma unroll
+        for (int t = 0; t < TOK_TILES; ++t) {
+          acc[t][0] = fmaf(s0, bacc[t][0], acc[t][0]);
+          acc[t][1] = fmaf(s0, bacc[t][1], acc[t][1]);
+          acc[t][2] = fmaf(s1, bacc[t][2], acc[t][2]);
+          acc[t][3] = fmaf(s1, bacc[t][3], acc[t][3]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[s]);
+    }
+    // Partial sums: rows lr0/lr1, tokens 2q, 2q+1 (+8t); red is [token][row].
+#pragma unroll
+    for (int t = 0; t < TOK_TILES; ++t) {
+      const int tok = 8 * t + 2 * q;
+      red[tok * kRows + lr0] = acc[t][0];
+      red[(tok + 1) * kRows + lr0] = acc[t][1];
+      red[tok * kRows + lr1] = acc[t][2];
+      red[(tok + 1) * kRows + lr1] = acc[t][3];
+    }
   }
+  __syncthreads();
   cluster_sync_all();
 
-  // Each CTA of the cluster finishes a slice of the 32 rows.
-  const int rpr = kRows / static_cast<int>(csize);
+  // Adapter intermediate T is written by the preceding kernel (a no-op when
+  // this grid was not launched as its programmatic dependent).
+  if (p.r > 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+  // CTA `crank` of the cluster finishes rows [r_lo, r_hi) of the tile.
+  const int r_lo = static_cast<int>((static_cast<uint32_t>(kRows) * crank) / csize);
+  const int r_hi = static_cast<int>((static_cast<uint32_t>(kRows) * (crank + 1)) / csize);
+  const int rpr = r_hi - r_lo;
   for (int i = threadIdx.x; i < p.m * rpr; i += kThreads) {
     const int mi = i / rpr;
-    const int nl = static_cast<int>(crank) * rpr + (i % rpr);
+    const int nl = r_lo + (i % rpr);
     const int64_t n = n_cta + nl;
     if (n >= p.n) continue;
-    float s = 0.f;
-    for (uint32_t peer = 0; peer < csize; ++peer) s += ld_dsmem_f32(&red[0][mi][nl], peer);
+    float sum = 0.f;
+    const uint32_t off = red_addr + static_cast<uint32_t>(mi * kRows + nl) * 4u;
+    for (uint32_t peer = 0; peer < csize; ++peer) sum += ld_dsmem_f32(off, peer);
     if (p.r > 0) {
       const uint16_t *trow = p.T + static_cast<int64_t>(mi) * p.r;
       const uint16_t *brow = p.B + n * p.r;
@@ -176,13 +352,12 @@ __global__ void __launch_bounds__(kThreads) gemv_fwd_kernel(const __grid_constan
         const uint32_t ba[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          s = fmaf(bf16lo_to_f32(ta[e]), bf16lo_to_f32(ba[e]), s);
-          s = fmaf(bf16hi_to_f32(ta[e]), bf16hi_to_f32(ba[e]), s);
+          sum = fmaf(bf16lo_to_f32(ta[e]), bf16lo_to_f32(ba[e]), sum);
+          sum = fmaf(bf16hi_to_f32(ta[e]), bf16hi_to_f32(ba[e]), sum);
         }
       }
     }
-    const uint32_t packed = pack_bf16x2(s, 0.f);
-    p.Y[static_cast<int64_t>(mi) * p.n + n] = static_cast<uint16_t>(packed & 0xFFFFu);
+    p.Y[static_cast<int64_t>(mi) * p.n + n] = static_cast<uint16_t>(pack_bf16x2(sum, 0.f) & 0xFFFFu);
   }
   cluster_sync_all();
 }
@@ -193,6 +368,9 @@ __global__ void __launch_bounds__(256) lora_proj_small_kernel(const uint16_t *__
                                                               int r, float scale,
                                                               uint16_t *__restrict__ T) {
   __shared__ float red[8][kMaxM];
+  // The weight-streaming kernel that consumes T may start now; it waits for
+  // this grid's completion before its epilogue reads T.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int j = blockIdx.x;
   const uint16_t *arow = A + static_cast<int64_t>(j) * k;
   float acc[kMaxM];
@@ -245,45 +423,70 @@ cudaError_t launch_lora_proj_small(const uint16_t *X, int64_t m, int64_t k, cons
 
 cudaError_t launch_gemv_fwd(const uint16_t *X, int64_t m, const uint8_t *codes, const uint8_t *absmax_q,
                             const float *group_scale, int64_t n, int64_t k, const uint16_t *T,
-                            const uint16_t *B, int32_t r, uint16_t *Y, cudaStream_t stream) {
+                            const uint16_t *B, int32_t r, uint16_t *Y, cudaStream_t stream, bool pdl) {
   if (m <= 0) return cudaSuccess;
   GemvParams p{};
+  if (!encode_codes_map(&p.tmCodes, codes, n, k / 2, 128, kRows, true)) return cudaErrorInvalidValue;
   p.X = X;
-  p.codes = codes;
   p.absmax_q = absmax_q;
   p.group_scale = group_scale;
   p.T = T;
   p.B = B;
   p.Y = Y;
+  p.err = device_error_word();
   p.n = n;
   p.k = k;
   p.m = static_cast<int>(m);
   p.r = (T != nullptr && B != nullptr) ? r : 0;
-  p.nchunks = static_cast<int>((k + 255) / 256);
   p.tab = nf4_tables();
 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static bool configured[64][2] = {};
+  const int variant = m <= 8 ? 0 : 1;
+  if (dev >= 0 && dev < 64 && !configured[dev][variant]) {
+    cudaError_t e = variant == 0
+                        ? cudaFuncSetAttribute(gemv_fwd_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(kSmemBytes))
+                        : cudaFuncSetAttribute(gemv_fwd_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(kSmemBytes));
+    if (e != cudaSuccess) return e;
+    configured[dev][variant] = true;
+  }
+  // Split K over a cluster of cs CTAs.  Pick cs in 1..8 to fill the resident
+  // CTA slots (two per SM) in as few, as full waves as possible, keeping at
+  // least two stages of K per CTA.
   const int64_t row_ctas = (n + kRows - 1) / kRows;
-  // Split K over a cluster until there are about three CTAs per SM, keeping
-  // at least one chunk of K per warp and never more than 8 CTAs per cluster.
+  const int64_t kblocks = k / 64;
+  const int64_t slots = 2LL * sms;
   int cs = 1;
-  while (cs < 8 && row_ctas * cs < 3LL * sms && p.nchunks / (cs * 2) >= kKParts) cs *= 2;
+  double best = -1.0;
+  for (int c = 1; c <= 8; ++c) {
+    if (c > 1 && (kblocks / kStageBlocks) / c < 2) break;
+    const int64_t ctas = row_ctas * c;
+    const int64_t waves = (ctas + slots - 1) / slots;
+    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
+    // Fuller waves first; among equal, fewer CTAs (less reduction traffic).
+    if (eff > best + 1e-9) { best = eff; cs = c; }
+  }
 
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(row_ctas), static_cast<unsigned>(cs), 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = static_cast<unsigned>(cs);
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_fwd_kernel, p);
+  cfg.numAttrs = (p.r > 0 && pdl) ? 2 : 1;
+  const cudaError_t e = variant == 0 ? cudaLaunchKernelEx(&cfg, gemv_fwd_kernel<1>, p)
+                                     : cudaLaunchKernelEx(&cfg, gemv_fwd_kernel<2>, p);
   if (e == cudaSuccess) count_launches(1);
   return e;
 }

@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "types.h"
@@ -22,6 +23,13 @@ void count_launches(int n);
 // qlora_last_cuda_error() and returns QLORA_ERR_CUDA.
 int status_from_cuda(cudaError_t e);
 
+// TMA tensor maps (2D, row-major).  bf16: 128-byte swizzle.  codes: uint8
+// rows of packed codes, optional 128-byte swizzle.  False if encoding failed.
+bool encode_bf16_map(CUtensorMap *m, const uint16_t *ptr, int64_t rows, int64_t cols, uint32_t box_cols,
+                     uint32_t box_rows);
+bool encode_codes_map(CUtensorMap *m, const uint8_t *ptr, int64_t rows, int64_t row_bytes, uint32_t box_bytes,
+                      uint32_t box_rows, bool swizzle128);
+
 // --- launchers (all asynchronous on `stream`; return cudaError_t) --------
 
 cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q,
@@ -34,11 +42,12 @@ cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *absmax_q, const 
 cudaError_t launch_lora_proj_small(const uint16_t *X, int64_t m, int64_t k, const uint16_t *A,
                                    int32_t r, float scale, uint16_t *T, cudaStream_t stream);
 
-// Y[m x n] = bf16(X . W^T + T . B^T) for m <= 16 (weight-streaming kernel).
+// Y[m x n] = bf16(X . W^T + T . B^T) for m <= 16 (weight-streaming kernel);
+// with pdl it overlaps the preceding T projection.
 cudaError_t launch_gemv_fwd(const uint16_t *X, int64_t m, const uint8_t *codes,
                             const uint8_t *absmax_q, const float *group_scale, int64_t n, int64_t k,
                             const uint16_t *T, const uint16_t *B, int32_t r, uint16_t *Y,
-                            cudaStream_t stream);
+                            cudaStream_t stream, bool pdl);
 
 // tcgen05 paths -------------------------------------------------------------
 
@@ -50,12 +59,15 @@ struct WeightView {
 };
 
 // Y = bf16(X . W^T + T . B^T); T may be null (no adapter).
+// With pdl, the kernel is launched as a programmatic dependent of the
+// preceding kernel (the adapter projection) and waits for it only before its
+// adapter k-steps.
 cudaError_t tc_fwd(const uint16_t *X, int64_t m, const WeightView &w, const uint16_t *T,
-                   const uint16_t *B, int32_t r, uint16_t *Y, cudaStream_t stream);
+                   const uint16_t *B, int32_t r, uint16_t *Y, cudaStream_t stream, bool pdl);
 
 // dX = bf16(dY . W^ + U . A); U may be null.
 cudaError_t tc_bwd_dx(const uint16_t *dY, int64_t m, const WeightView &w, const uint16_t *U,
-                      const uint16_t *A, int32_t r, uint16_t *dX, cudaStream_t stream);
+                      const uint16_t *A, int32_t r, uint16_t *dX, cudaStream_t stream, bool pdl);
 
 // out[m x r] = bf16(scale * L[m x kc] . R^T) with R given as [r x kc] (k-major).
 cudaError_t tc_proj_kmajor(const uint16_t *L, int64_t m, int64_t kc, const uint16_t *R, int32_t r,

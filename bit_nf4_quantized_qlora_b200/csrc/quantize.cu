@@ -6,11 +6,12 @@
 // constants are themselves quantized to 8 bits in blocks of 256.
 //
 // One CTA of 256 threads per group of 256 blocks (16384 weights, 64 KB of
-// fp32).  Each warp owns 32 blocks and reads them as 16 coalesced 512-byte
-// rows (two blocks per row, 16 lanes per block, one float4 per lane); the
-// block absmax is a 16-lane shuffle reduction, the codes are counted against
-// the 15 fp32 midpoints after an IEEE division by the absmax, and each lane
-// stores its 4 codes as one 16-bit word.  The group maximum is then reduced
+// fp32).  Each warp owns 32 blocks; four lanes share a block and each holds 16
+// of its weights, so a lane has 16 independent division + search chains in
+// flight.  The block absmax is a 4-lane shuffle reduction; each weight is
+// divided by it (correctly rounded, see div_by_absmax) and located among the
+// 15 fp32 midpoints by a branchless binary search; codes are stored as 16-bit
+// words (4 weights).  The group maximum is then reduced
 // through shared memory and every thread emits one absmax code.
 #include "common.cuh"
 #include "internal.h"
@@ -22,11 +23,27 @@ constexpr int kThreads = 256;
 constexpr int kBlocksPerGroup = 256;
 constexpr int kUnroll = 4;
 
-__device__ __forceinline__ uint32_t nf4_code(float x, const Nf4Tables &tab) {
-  uint32_t c = 0;
-#pragma unroll
-  for (int i = 0; i < 15; ++i) c += (x > tab.mid[i]) ? 1u : 0u;
-  return c;
+// Absmax values below this take the IEEE division path (1/m stays finite and
+// normal far above it).
+constexpr float kMinFastAbsmax = 0x1p-100f;
+
+__device__ __forceinline__ float div_by_absmax(float w, float m, float y) {
+  const float q0 = __fmul_rn(w, y);
+  const float rho = __fmaf_rn(-q0, m, w);
+  return __fmaf_rn(rho, y, q0);
+}
+
+// #{i : x > T_i} over the 15 sorted midpoints, as a branchless binary search:
+// code >= 8 iff x > T7; then code >= base + 4 iff x > T[base + 3], and so on.
+__device__ __forceinline__ uint32_t nf4_code(float x, const Nf4Tables &t) {
+  const bool b3 = x > t.mid[7];
+  const bool b2 = x > (b3 ? t.mid[11] : t.mid[3]);
+  const float m1 = b2 ? (b3 ? t.mid[13] : t.mid[5]) : (b3 ? t.mid[9] : t.mid[1]);
+  const bool b1 = x > m1;
+  const float lo = b1 ? (b3 ? t.mid[10] : t.mid[2]) : (b3 ? t.mid[8] : t.mid[0]);
+  const float hi = b1 ? (b3 ? t.mid[14] : t.mid[6]) : (b3 ? t.mid[12] : t.mid[4]);
+  const bool b0 = x > (b2 ? hi : lo);
+  return (b3 ? 8u : 0u) | (b2 ? 4u : 0u) | (b1 ? 2u : 0u) | (b0 ? 1u : 0u);
 }
 
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const float *__restrict__ W, int64_t nb,
@@ -43,43 +60,77 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const float *__restr
   const int nblk = static_cast<int>(nb - b0 < kBlocksPerGroup ? nb - b0 : kBlocksPerGroup);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int half = lane >> 4;   // which of the two blocks of a 512-byte row
-  const int sub = lane & 15;    // float4 index inside the block
+  const int sub = lane & 3;      // 4 lanes per block, 16 weights each
+  const int bl = lane >> 2;      // 8 blocks per warp iteration
 
-  // Warp w owns blocks [32w, 32w + 32) of the group: 16 rows of 2 blocks.
-#pragma unroll 1
-  for (int j0 = 0; j0 < 16; j0 += kUnroll) {
-    float4 v[kUnroll];
+  // Warp w owns blocks [32w, 32w + 32): 4 iterations of 8 blocks.  Lane
+  // (bl, sub) holds weights 16j + 4sub .. +3 (j = 0..3) of its block, so each
+  // load instruction reads 8 blocks x 64 contiguous bytes.
+  float4 v[4], nv[4];
+  auto load = [&](int it, float4 (&dst)[4]) {
+    const int blk = warp * 32 + it * 8 + bl;
+    if (blk < nblk) {
+      const float4 *src = reinterpret_cast<const float4 *>(W + (b0 + blk) * 64) + sub;
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int blk = warp * 32 + 2 * (j0 + u) + half;
-      if (blk < nblk) {
-        v[u] = __ldcs(reinterpret_cast<const float4 *>(W + (b0 + blk) * 64) + sub);
+      for (int j = 0; j < 4; ++j) dst[j] = __ldcs(src + 4 * j);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) dst[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  load(0, v);
+#pragma unroll 1
+  for (int it = 0; it < 4; ++it) {
+    if (it + 1 < 4) load(it + 1, nv);
+    const int blk = warp * 32 + it * 8 + bl;
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(v[j].x), fabsf(v[j].y)), fmaxf(fabsf(v[j].z), fabsf(v[j].w))));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    if (blk < nblk) {
+      uint32_t c[16];
+      if (m >= kMinFastAbsmax) {
+        // Correctly rounded w / m without a divide per weight (Markstein's
+        // theorem): with y = RN(1/m) and q0 = RN(w*y) within one ulp of w/m,
+        // the residual w - m*q0 is exact in one FMA and RN(q0 + residual*y)
+        // is RN(w/m).  |w/m| <= 1 cannot overflow; results below the normal
+        // range all give code 7, where rounding does not matter.
+        const float y = __frcp_rn(m);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          c[4 * j + 0] = nf4_code(div_by_absmax(v[j].x, m, y), tab);
+          c[4 * j + 1] = nf4_code(div_by_absmax(v[j].y, m, y), tab);
+          c[4 * j + 2] = nf4_code(div_by_absmax(v[j].z, m, y), tab);
+          c[4 * j + 3] = nf4_code(div_by_absmax(v[j].w, m, y), tab);
+        }
+      } else if (m > 0.0f) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          c[4 * j + 0] = nf4_code(__fdiv_rn(v[j].x, m), tab);
+          c[4 * j + 1] = nf4_code(__fdiv_rn(v[j].y, m), tab);
+          c[4 * j + 2] = nf4_code(__fdiv_rn(v[j].z, m), tab);
+          c[4 * j + 3] = nf4_code(__fdiv_rn(v[j].w, m), tab);
+        }
       } else {
-        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) c[e] = 7u;
+      }
+      uint16_t *dst = reinterpret_cast<uint16_t *>(codes + (b0 + blk) * 32);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t packed = ((c[4 * j] << 4) | c[4 * j + 1]) | (((c[4 * j + 2] << 4) | c[4 * j + 3]) << 8);
+        dst[4 * j + sub] = static_cast<uint16_t>(packed);      // bytes 8j + 2sub, +1
+      }
+      if (sub == 0) {
+        s_c[blk] = m;
+        if (absmax_out) absmax_out[b0 + blk] = m;
       }
     }
+    if (it + 1 < 4) {
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int blk = warp * 32 + 2 * (j0 + u) + half;
-      float m = fmaxf(fmaxf(fabsf(v[u].x), fabsf(v[u].y)), fmaxf(fabsf(v[u].z), fabsf(v[u].w)));
-#pragma unroll
-      for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if (blk < nblk) {
-        uint32_t c0 = 7, c1 = 7, c2 = 7, c3 = 7;
-        if (m > 0.0f) {
-          c0 = nf4_code(__fdiv_rn(v[u].x, m), tab);
-          c1 = nf4_code(__fdiv_rn(v[u].y, m), tab);
-          c2 = nf4_code(__fdiv_rn(v[u].z, m), tab);
-          c3 = nf4_code(__fdiv_rn(v[u].w, m), tab);
-        }
-        const uint32_t packed = ((c0 << 4) | c1) | (((c2 << 4) | c3) << 8);
-        reinterpret_cast<uint16_t *>(codes + (b0 + blk) * 32)[sub] = static_cast<uint16_t>(packed);
-        if (sub == 0) {
-          s_c[blk] = m;
-          if (absmax_out) absmax_out[b0 + blk] = m;
-        }
-      }
+      for (int j = 0; j < 4; ++j) v[j] = nv[j];
     }
   }
   __syncthreads();

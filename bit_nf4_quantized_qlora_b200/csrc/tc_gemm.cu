@@ -60,6 +60,7 @@ struct __align__(64) TcParams {
   int64_t out_ld;
   int out_rows, out_cols;
   int num_main, num_lora;
+  int pdl;              // launched as a programmatic dependent of the adapter projection
   float alpha;
   Nf4Tables tab;
 };
@@ -132,8 +133,9 @@ __device__ __forceinline__ void sts128(uint32_t addr, const uint32_t (&v)[4]) {
 
 // ---- compile-time configuration -------------------------------------------
 
-template <int BN_, int MSUB_, bool A_MN_, bool B_NF4_, bool B_MN_, bool OUT_T_>
+template <int BN_, int MSUB_, bool A_MN_, bool B_NF4_, bool B_MN_, bool OUT_T_, bool SPLIT_ = false>
 struct Cfg {
+  static constexpr bool SPLIT = SPLIT_;   // K split over a cluster, DSMEM reduction
   static constexpr int BN = BN_;
   static constexpr int MSUB = MSUB_;
   static constexpr bool A_MN = A_MN_;
@@ -146,9 +148,13 @@ struct Cfg {
   static constexpr uint32_t CODE_BYTES = B_NF4 ? static_cast<uint32_t>(BN) * 32u : 0u;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + CODE_BYTES;
   static constexpr int STAGES_RAW = static_cast<int>((224u * 1024u) / STAGE_BYTES);
-  static constexpr int STAGES = STAGES_RAW > 6 ? 6 : STAGES_RAW;
+  // Skinny (BN=64) configs keep 4 stages so two CTAs fit on an SM.
+  static constexpr int STAGES = B_NF4 ? (STAGES_RAW > 6 ? 6 : STAGES_RAW) : 4;
   static constexpr uint32_t SMEM_BYTES = STAGE_BYTES * STAGES + 1024u;
-  static constexpr int NUM_EPI_WARPS = B_NF4 ? 8 : 4;
+  // NF4 modes: groups of 8 dequant warps take k-steps in turn (two groups for
+  // the K-major forward tile, one for the MN-major input-gradient tile).
+  static constexpr int DQ_GROUPS = B_NF4 ? (B_MN ? 1 : 2) : 0;
+  static constexpr int NUM_EPI_WARPS = B_NF4 ? 8 * DQ_GROUPS : 4;
   static constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
   static constexpr uint32_t TMEM_RAW = static_cast<uint32_t>(BN * MSUB);
   static constexpr uint32_t TMEM_COLS = TMEM_RAW <= 32 ? 32 : TMEM_RAW <= 64 ? 64 : TMEM_RAW <= 128 ? 128 : TMEM_RAW <= 256 ? 256 : 512;
@@ -157,7 +163,30 @@ struct Cfg {
   static_assert(!(A_MN && MSUB != 1), "MN-major A supports one 128-row tile");
   static_assert(!B_NF4 || BN == 256, "NF4 modes use 256-wide tiles (one block per dequant thread)");
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
+  static_assert(!SPLIT || (!B_NF4 && MSUB == 1 && BN == 64), "split-K is for the skinny products");
+  static_assert(!SPLIT || STAGE_BYTES * STAGES >= 128u * 64u * 4u, "room for the fp32 partial tile");
 };
+
+__device__ __forceinline__ uint32_t cl_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cl_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cl_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float ld_peer_f32(uint32_t local_addr, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
 
 template <class C>
 __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_constant__ TcParams p) {
@@ -174,12 +203,22 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
   const int lane = threadIdx.x & 31;
   const int n_tile = blockIdx.x;
   const int m_tile = blockIdx.y;
-  const int total = p.num_main + p.num_lora;
+  // With split-K, CTA z of the cluster runs k-steps [it_begin, it_end).
+  int it_begin = 0, total = p.num_main + p.num_lora;
+  if (C::SPLIT) {
+    const int z = static_cast<int>(blockIdx.z), nz = static_cast<int>(gridDim.z);
+    it_begin = static_cast<int>((static_cast<int64_t>(p.num_main) * z) / nz);
+    total = static_cast<int>((static_cast<int64_t>(p.num_main) * (z + 1)) / nz);
+  }
+  const int n_iters = total - it_begin;
 
+  // A skinny projection lets the kernel that consumes its output launch now;
+  // that kernel waits for this grid before it reads the output.
+  if (C::SPLIT) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full_a[s], 1);
-      mbar_init(&full_b[s], C::B_NF4 ? 8 : 1);
+      mbar_init(&full_b[s], C::B_NF4 ? 8 : 1);   // one group of 8 dequant warps per stage fill
       mbar_init(&empty_bar[s], 1);
     }
     mbar_init(&acc_bar, 1);
@@ -202,9 +241,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int issued = 0;
-      for (int it = 0; it < total; ++it) {
-        const int s = it % C::STAGES;
-        const uint32_t ph = static_cast<uint32_t>(it / C::STAGES) & 1u;
+      for (int it = it_begin; it < total; ++it) {
+        const int li = it - it_begin;
+        const int s = li % C::STAGES;
+        const uint32_t ph = static_cast<uint32_t>(li / C::STAGES) & 1u;
         if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, p.err, kErrTimeoutEmpty)) break;
         const uint32_t a_s = base + static_cast<uint32_t>(s) * C::STAGE_BYTES;
         const uint32_t b_s = a_s + C::A_BYTES;
@@ -239,6 +279,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
           }
         } else {
           const int l = it - p.num_main;
+          // The adapter operand comes from the preceding projection kernel.
+          if (l == 0 && p.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
           mbar_arrive_expect_tx(&full_a[s], C::A_BYTES + C::B_BYTES);
 #pragma unroll
           for (int h = 0; h < C::MSUB; ++h)
@@ -262,9 +304,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = true;
-      for (int it = 0; it < total && ok; ++it) {
-        const int s = it % C::STAGES;
-        const uint32_t ph = static_cast<uint32_t>(it / C::STAGES) & 1u;
+      for (int it = it_begin; it < total && ok; ++it) {
+        const int li = it - it_begin;
+        const int s = li % C::STAGES;
+        const uint32_t ph = static_cast<uint32_t>(li / C::STAGES) & 1u;
         ok = mbar_wait_bounded(&full_a[s], ph, p.err, kErrTimeoutFullA);
         if (ok && C::B_NF4) ok = mbar_wait_bounded(&full_b[s], ph, p.err, kErrTimeoutFullB);
         if (!ok) break;
@@ -279,7 +322,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
                                         : smem_desc(a_s + h * kASub + kk * 32u, 16u, 1024u);
             const uint64_t bd = C::B_MN ? smem_desc(b_s + kk * 2048u, 8192u, 1024u)
                                         : smem_desc(b_s + kk * 32u, 16u, 1024u);
-            umma_f16(tmem + static_cast<uint32_t>(h * C::BN), ad, bd, C::IDESC, (it > 0 || kk > 0) ? 1u : 0u);
+            umma_f16(tmem + static_cast<uint32_t>(h * C::BN), ad, bd, C::IDESC, (li > 0 || kk > 0) ? 1u : 0u);
           }
         }
         umma_commit(&empty_bar[s]);
@@ -288,7 +331,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
     }
   } else {
     // ------------------------------------------------------------ dequant
-    const int dt = threadIdx.x - 64;  // 0 .. 32*NUM_EPI_WARPS-1
+    // Groups of 8 warps take k-steps in turn, so DQ_GROUPS B tiles are being
+    // expanded at once; within a group thread dt fills one 128-byte row.
+    const int grp = (warp - 2) >> 3;                 // 0 .. DQ_GROUPS-1 (NF4 modes)
+    const int dt = (threadIdx.x - 64) & 255;
     bool ok = true;
     if (C::B_NF4) {
       const int64_t kblocks = p.w_k / 64;
@@ -312,16 +358,17 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
         }
         return (gn < p.w_n && kb < kblocks) ? gn * kblocks + kb : -1;
       };
-      // The absmax code and group constant of the next step are fetched one
-      // step ahead so their latency hides behind the current decode.
-      int64_t blk_nx = p.num_main > 0 ? block_of(0) : -1;
-      uint32_t q_nx = 0;
-      float S_nx = 0.f;
-      if (blk_nx >= 0) {
-        q_nx = __ldg(p.absmax_q + blk_nx);
-        S_nx = __ldg(p.group_scale + (blk_nx >> 8));
-      }
-      for (int it = 0; it < total; ++it) {
+      // Absmax code and group constant of this group's next step, fetched one
+      // step of the group (DQ_GROUPS k-steps) ahead.  The group constant
+      // t = fp32(S / 255) is recomputed only when the group index changes
+      // (in the forward a thread walks one weight row, so that is rare).
+      int64_t blk_nx = grp < p.num_main ? block_of(grp) : -1;
+      uint32_t q_nx = blk_nx >= 0 ? __ldg(p.absmax_q + blk_nx) : 0u;
+      float S_nx = blk_nx >= 0 ? __ldg(p.group_scale + (blk_nx >> 8)) : 0.f;
+      int64_t g_cur = -1;
+      float t_cur = 0.f;
+      constexpr int kStride = C::DQ_GROUPS > 0 ? C::DQ_GROUPS : 1;
+      for (int it = grp; it < total; it += kStride) {
         const int s = it % C::STAGES;
         const uint32_t ph = static_cast<uint32_t>(it / C::STAGES) & 1u;
         if (!mbar_wait_bounded(&full_a[s], ph, p.err, kErrTimeoutFullA)) { ok = false; break; }
@@ -329,12 +376,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
           const int64_t blk = blk_nx;
           const uint32_t qv = q_nx;
           const float S = S_nx;
-          if (it + 1 < p.num_main) {
-            blk_nx = block_of(it + 1);
-            if (blk_nx >= 0) {
-              q_nx = __ldg(p.absmax_q + blk_nx);
-              S_nx = __ldg(p.group_scale + (blk_nx >> 8));
-            }
+          if (it + kStride < p.num_main) {
+            blk_nx = block_of(it + kStride);
+            q_nx = blk_nx >= 0 ? __ldg(p.absmax_q + blk_nx) : 0u;
+            S_nx = blk_nx >= 0 ? __ldg(p.group_scale + (blk_nx >> 8)) : 0.f;
           }
           const uint32_t a_s = base + static_cast<uint32_t>(s) * C::STAGE_BYTES;
           const uint32_t b_s = a_s + C::A_BYTES;
@@ -342,11 +387,16 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
           Bf16Table tb;
           uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = make_uint4(0u, 0u, 0u, 0u);
           if (blk >= 0) {
+            const int64_t gi = blk >> 8;
+            if (gi != g_cur) {
+              g_cur = gi;
+              t_cur = __fdiv_rn(S, 255.0f);
+            }
             const uint4 f = lds128(c_s + code_off + first_half);
             const uint4 g2 = lds128(c_s + code_off + (16u - first_half));
             lo = first_half ? g2 : f;
             hi = first_half ? f : g2;
-            make_table(p.tab, absmax_dequant(qv, S), tb);
+            make_table(p.tab, __fmul_rn(static_cast<float>(qv), t_cur), tb);
           } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j) tb.lo[j] = tb.hi[j] = 0u;
@@ -380,6 +430,17 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
           c_begin = (ew >> 2) * (C::BN / 2);
           c_end = c_begin + C::BN / 2;
         }
+      } else if (C::NUM_EPI_WARPS == 16) {
+        // 16 warps: 4 lane quadrants x (accumulator half, column half) or
+        // x column quarter.
+        if (C::MSUB == 2) {
+          h = ew >> 3;
+          c_begin = ((ew >> 2) & 1) * (C::BN / 2);
+          c_end = c_begin + C::BN / 2;
+        } else {
+          c_begin = (ew >> 2) * (C::BN / 4);
+          c_end = c_begin + C::BN / 4;
+        }
       }
       const int row_in_tile = h * 128 + quad * 32 + lane;
       const int64_t grow = static_cast<int64_t>(m_tile) * C::BM + row_in_tile;
@@ -387,6 +448,16 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
       for (int c0 = c_begin; c0 < c_end; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(h * C::BN + c0), v);
+        if (C::SPLIT) {
+          // fp32 partial, column-major [col][row] in this CTA's idle stage memory.
+          const uint32_t dst = base + (static_cast<uint32_t>(c0) * 128u + static_cast<uint32_t>(row_in_tile)) * 4u;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float val = n_iters > 0 ? __uint_as_float(v[j]) : 0.f;
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(dst + static_cast<uint32_t>(j) * 512u), "f"(val) : "memory");
+          }
+          continue;
+        }
         const int64_t gcol = static_cast<int64_t>(n_tile) * C::BN + c0;
         if (!C::OUT_T) {
           if (row_ok) {
@@ -421,6 +492,30 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
 
   tc_fence_before();
   __syncthreads();
+  if (C::SPLIT) {
+    // Reduce the cluster's partial tiles through distributed shared memory:
+    // CTA `rank` finishes rows [rank*128/size, (rank+1)*128/size).
+    cl_sync();
+    const uint32_t rank = cl_rank(), size = cl_size();
+    const int r_lo = static_cast<int>((128u * rank) / size), r_hi = static_cast<int>((128u * (rank + 1)) / size);
+    const int rows = r_hi - r_lo;
+    for (int i = threadIdx.x; i < rows * C::BN; i += C::NUM_THREADS) {
+      const int col = i / rows, row = r_lo + (i % rows);
+      const uint32_t off = base + (static_cast<uint32_t>(col) * 128u + static_cast<uint32_t>(row)) * 4u;
+      float acc = 0.f;
+      for (uint32_t pr = 0; pr < size; ++pr) acc += ld_peer_f32(off, pr);
+      const int64_t grow = static_cast<int64_t>(m_tile) * C::BM + row;
+      const int64_t gcol = static_cast<int64_t>(n_tile) * C::BN + col;
+      if (grow < p.out_rows && gcol < p.out_cols) {
+        const uint16_t v = static_cast<uint16_t>(pack_bf16x2(acc * p.alpha, 0.f) & 0xFFFFu);
+        if (C::OUT_T) p.out[gcol * p.out_ld + grow] = v;
+        else p.out[grow * p.out_ld + gcol] = v;
+      }
+    }
+    cl_sync();
+  }
+  tc_fence_before();
+  __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS) : "memory");
@@ -429,51 +524,9 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
 
 // ---- host side ------------------------------------------------------------
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void *f = nullptr;
-    cudaDriverEntryPointQueryResult q{};
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-  }
-  return fn;
-}
-
-// 2D map over a row-major [outer x inner] tensor with a row pitch in bytes.
-bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint64_t inner, uint64_t outer,
-              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t es[2] = {1, 1};
-  return fn(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-bool map_bf16(CUtensorMap *m, const uint16_t *ptr, int64_t rows, int64_t cols, uint32_t box_cols, uint32_t box_rows) {
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, static_cast<uint64_t>(cols), static_cast<uint64_t>(rows),
-                  static_cast<uint64_t>(cols) * 2u, box_cols, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
-}
-
-bool map_codes(CUtensorMap *m, const uint8_t *ptr, int64_t rows, int64_t row_bytes, uint32_t box_bytes,
-               uint32_t box_rows) {
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, ptr, static_cast<uint64_t>(row_bytes),
-                  static_cast<uint64_t>(rows), static_cast<uint64_t>(row_bytes), box_bytes, box_rows,
-                  CU_TENSOR_MAP_SWIZZLE_NONE);
-}
-
 template <class C>
-cudaError_t launch(const TcParams &p, int grid_n, int grid_m, cudaStream_t stream) {
+cudaError_t launch(const TcParams &p, int grid_n, int grid_m, cudaStream_t stream, int split = 1,
+                   bool pdl = false) {
   static bool configured[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -485,9 +538,44 @@ cudaError_t launch(const TcParams &p, int grid_n, int grid_m, cudaStream_t strea
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
   if (grid_n <= 0 || grid_m <= 0) return cudaSuccess;
-  tc_kernel<C><<<dim3(grid_n, grid_m, 1), C::NUM_THREADS, C::SMEM_BYTES, stream>>>(p);
-  count_launches(1);
-  return cudaGetLastError();
+  if (split < 1 || !C::SPLIT) split = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid_n, grid_m, split);
+  cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (C::SPLIT) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = static_cast<unsigned>(split);
+    ++na;
+  }
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = na ? attr : nullptr;
+  cfg.numAttrs = na;
+  e = cudaLaunchKernelEx(&cfg, tc_kernel<C>, p);
+  if (e == cudaSuccess) count_launches(1);
+  return e;
+}
+
+// Split of the contraction for a skinny product with `tiles` output tiles and
+// `ksteps` k-steps: fill about two CTAs per SM, at least two k-steps per CTA,
+// at most 8 CTAs per cluster.
+int choose_split(int64_t tiles, int ksteps) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t sp = (2LL * sms) / (tiles > 0 ? tiles : 1);
+  if (sp > 8) sp = 8;
+  if (sp > ksteps / 2) sp = ksteps / 2;
+  return sp < 1 ? 1 : static_cast<int>(sp);
 }
 
 int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
@@ -496,24 +584,24 @@ using CfgFwd2 = Cfg<256, 2, false, true, false, false>;
 using CfgFwd1 = Cfg<256, 1, false, true, false, false>;
 using CfgBwd2 = Cfg<256, 2, false, true, true, false>;
 using CfgBwd1 = Cfg<256, 1, false, true, true, false>;
-using CfgProjK = Cfg<64, 1, false, false, false, false>;
-using CfgProjMN = Cfg<64, 1, false, false, true, false>;
-using CfgTN = Cfg<64, 1, true, false, true, false>;
-using CfgTNT = Cfg<64, 1, true, false, true, true>;
+using CfgProjK = Cfg<64, 1, false, false, false, false, true>;
+using CfgProjMN = Cfg<64, 1, false, false, true, false, true>;
+using CfgTN = Cfg<64, 1, true, false, true, false, true>;
+using CfgTNT = Cfg<64, 1, true, false, true, true, true>;
 
 }  // namespace
 
 cudaError_t tc_fwd(const uint16_t *X, int64_t m, const WeightView &w, const uint16_t *T, const uint16_t *B,
-                   int32_t r, uint16_t *Y, cudaStream_t stream) {
+                   int32_t r, uint16_t *Y, cudaStream_t stream, bool pdl) {
   TcParams p{};
   const bool big = m > 128;
   const uint32_t bm = big ? 256u : 128u;
   const bool lora = T != nullptr && B != nullptr && r > 0;
-  if (!map_bf16(&p.tmA, X, m, w.k, 64, 128)) return cudaErrorInvalidValue;
-  if (!map_codes(&p.tmCodes, w.codes, w.n, w.k / 2, 32, 256)) return cudaErrorInvalidValue;
+  if (!encode_bf16_map(&p.tmA, X, m, w.k, 64, 128)) return cudaErrorInvalidValue;
+  if (!encode_codes_map(&p.tmCodes, w.codes, w.n, w.k / 2, 32, 256, false)) return cudaErrorInvalidValue;
   if (lora) {
-    if (!map_bf16(&p.tmA2, T, m, r, 64, 128)) return cudaErrorInvalidValue;
-    if (!map_bf16(&p.tmB2, B, w.n, r, 64, 256)) return cudaErrorInvalidValue;
+    if (!encode_bf16_map(&p.tmA2, T, m, r, 64, 128)) return cudaErrorInvalidValue;
+    if (!encode_bf16_map(&p.tmB2, B, w.n, r, 64, 256)) return cudaErrorInvalidValue;
   }
   p.absmax_q = w.absmax_q;
   p.group_scale = w.group_scale;
@@ -526,23 +614,25 @@ cudaError_t tc_fwd(const uint16_t *X, int64_t m, const WeightView &w, const uint
   p.out_cols = static_cast<int>(w.n);
   p.num_main = static_cast<int>(w.k / 64);
   p.num_lora = lora ? cdiv(r, 64) : 0;
+  p.pdl = (lora && pdl) ? 1 : 0;
   p.alpha = 1.0f;
   p.tab = nf4_tables();
   const int gn = cdiv(w.n, 256), gm = cdiv(m, bm);
-  return big ? launch<CfgFwd2>(p, gn, gm, stream) : launch<CfgFwd1>(p, gn, gm, stream);
+  return big ? launch<CfgFwd2>(p, gn, gm, stream, 1, p.pdl != 0)
+             : launch<CfgFwd1>(p, gn, gm, stream, 1, p.pdl != 0);
 }
 
 cudaError_t tc_bwd_dx(const uint16_t *dY, int64_t m, const WeightView &w, const uint16_t *U, const uint16_t *A,
-                      int32_t r, uint16_t *dX, cudaStream_t stream) {
+                      int32_t r, uint16_t *dX, cudaStream_t stream, bool pdl) {
   TcParams p{};
   const bool big = m > 128;
   const uint32_t bm = big ? 256u : 128u;
   const bool lora = U != nullptr && A != nullptr && r > 0;
-  if (!map_bf16(&p.tmA, dY, m, w.n, 64, 128)) return cudaErrorInvalidValue;
-  if (!map_codes(&p.tmCodes, w.codes, w.n, w.k / 2, 32, 64)) return cudaErrorInvalidValue;
+  if (!encode_bf16_map(&p.tmA, dY, m, w.n, 64, 128)) return cudaErrorInvalidValue;
+  if (!encode_codes_map(&p.tmCodes, w.codes, w.n, w.k / 2, 32, 64, false)) return cudaErrorInvalidValue;
   if (lora) {
-    if (!map_bf16(&p.tmA2, U, m, r, 64, 128)) return cudaErrorInvalidValue;
-    if (!map_bf16(&p.tmB2, A, r, w.k, 64, 64)) return cudaErrorInvalidValue;
+    if (!encode_bf16_map(&p.tmA2, U, m, r, 64, 128)) return cudaErrorInvalidValue;
+    if (!encode_bf16_map(&p.tmB2, A, r, w.k, 64, 64)) return cudaErrorInvalidValue;
   }
   p.absmax_q = w.absmax_q;
   p.group_scale = w.group_scale;
@@ -555,17 +645,19 @@ cudaError_t tc_bwd_dx(const uint16_t *dY, int64_t m, const WeightView &w, const 
   p.out_cols = static_cast<int>(w.k);
   p.num_main = cdiv(w.n, 64);
   p.num_lora = lora ? cdiv(r, 64) : 0;
+  p.pdl = (lora && pdl) ? 1 : 0;
   p.alpha = 1.0f;
   p.tab = nf4_tables();
   const int gn = cdiv(w.k, 256), gm = cdiv(m, bm);
-  return big ? launch<CfgBwd2>(p, gn, gm, stream) : launch<CfgBwd1>(p, gn, gm, stream);
+  return big ? launch<CfgBwd2>(p, gn, gm, stream, 1, p.pdl != 0)
+             : launch<CfgBwd1>(p, gn, gm, stream, 1, p.pdl != 0);
 }
 
 cudaError_t tc_proj_kmajor(const uint16_t *L, int64_t m, int64_t kc, const uint16_t *R, int32_t r, float scale,
                            uint16_t *out, cudaStream_t stream) {
   TcParams p{};
-  if (!map_bf16(&p.tmA, L, m, kc, 64, 128)) return cudaErrorInvalidValue;
-  if (!map_bf16(&p.tmB, R, r, kc, 64, 64)) return cudaErrorInvalidValue;
+  if (!encode_bf16_map(&p.tmA, L, m, kc, 64, 128)) return cudaErrorInvalidValue;
+  if (!encode_bf16_map(&p.tmB, R, r, kc, 64, 64)) return cudaErrorInvalidValue;
   p.out = out;
   p.err = device_error_word();
   p.out_ld = r;
@@ -574,14 +666,15 @@ cudaError_t tc_proj_kmajor(const uint16_t *L, int64_t m, int64_t kc, const uint1
   p.num_main = cdiv(kc, 64);
   p.num_lora = 0;
   p.alpha = scale;
-  return launch<CfgProjK>(p, cdiv(r, 64), cdiv(m, 128), stream);
+  const int gn = cdiv(r, 64), gm = cdiv(m, 128);
+  return launch<CfgProjK>(p, gn, gm, stream, choose_split(int64_t(gn) * gm, p.num_main));
 }
 
 cudaError_t tc_proj_mnmajor(const uint16_t *L, int64_t m, int64_t kc, const uint16_t *R, int32_t r, float scale,
                             uint16_t *out, cudaStream_t stream) {
   TcParams p{};
-  if (!map_bf16(&p.tmA, L, m, kc, 64, 128)) return cudaErrorInvalidValue;
-  if (!map_bf16(&p.tmB, R, kc, r, 64, 64)) return cudaErrorInvalidValue;
+  if (!encode_bf16_map(&p.tmA, L, m, kc, 64, 128)) return cudaErrorInvalidValue;
+  if (!encode_bf16_map(&p.tmB, R, kc, r, 64, 64)) return cudaErrorInvalidValue;
   p.out = out;
   p.err = device_error_word();
   p.out_ld = r;
@@ -590,14 +683,15 @@ cudaError_t tc_proj_mnmajor(const uint16_t *L, int64_t m, int64_t kc, const uint
   p.num_main = cdiv(kc, 64);
   p.num_lora = 0;
   p.alpha = scale;
-  return launch<CfgProjMN>(p, cdiv(r, 64), cdiv(m, 128), stream);
+  const int gn = cdiv(r, 64), gm = cdiv(m, 128);
+  return launch<CfgProjMN>(p, gn, gm, stream, choose_split(int64_t(gn) * gm, p.num_main));
 }
 
 cudaError_t tc_tn_skinny(const uint16_t *Lt, int64_t mc, int64_t pdim, const uint16_t *R, int32_t r, uint16_t *out,
                          bool transposed, cudaStream_t stream) {
   TcParams p{};
-  if (!map_bf16(&p.tmA, Lt, mc, pdim, 64, 64)) return cudaErrorInvalidValue;
-  if (!map_bf16(&p.tmB, R, mc, r, 64, 64)) return cudaErrorInvalidValue;
+  if (!encode_bf16_map(&p.tmA, Lt, mc, pdim, 64, 64)) return cudaErrorInvalidValue;
+  if (!encode_bf16_map(&p.tmB, R, mc, r, 64, 64)) return cudaErrorInvalidValue;
   p.out = out;
   p.err = device_error_word();
   p.out_ld = transposed ? pdim : r;
@@ -606,8 +700,9 @@ cudaError_t tc_tn_skinny(const uint16_t *Lt, int64_t mc, int64_t pdim, const uin
   p.num_main = cdiv(mc, 64);
   p.num_lora = 0;
   p.alpha = 1.0f;
-  return transposed ? launch<CfgTNT>(p, cdiv(r, 64), cdiv(pdim, 128), stream)
-                    : launch<CfgTN>(p, cdiv(r, 64), cdiv(pdim, 128), stream);
+  const int gn = cdiv(r, 64), gm = cdiv(pdim, 128);
+  const int sp = choose_split(int64_t(gn) * gm, p.num_main);
+  return transposed ? launch<CfgTNT>(p, gn, gm, stream, sp) : launch<CfgTN>(p, gn, gm, stream, sp);
 }
 
 }  // namespace qlora

@@ -56,6 +56,36 @@ def test_quantize_bit_exact(shape):
     assert np.array_equal(_np(w.group_scale).view(np.uint32), S.view(np.uint32))
 
 
+def test_quantize_codes_near_midpoints():
+    """Weights on and within +-2 ulps of every midpoint times the block absmax,
+    for 2048 random absmax values spanning 40 binades: the codes must equal the
+    oracle's, which divides with IEEE round-to-nearest."""
+    from oracle import nf4 as onf4
+    rng = np.random.default_rng(42)
+    mids = onf4.midpoints_f32()
+    nblk = 2048
+    c = (2.0 ** rng.uniform(-30, 10, nblk)).astype(np.float32)
+    W = np.zeros((nblk, 64), dtype=np.float32)
+    W[:, 0] = c                                       # the absmax element
+    for b in range(nblk):
+        vals = []
+        for t in mids:
+            base = np.float32(t * c[b])
+            for d in (-2, -1, 0, 1, 2):
+                v = base
+                for _ in range(abs(d)):
+                    v = np.nextafter(v, np.float32(np.inf if d > 0 else -np.inf))
+                vals.append(v)
+        vals = np.roll(np.array(vals, dtype=np.float32), -5 * (b % 15))[:63]   # all midpoints over 15 blocks
+        vals = np.clip(vals, -c[b], c[b])
+        W[b, 1:1 + len(vals)] = vals
+    Wt = torch.from_numpy(W.reshape(256, 512))
+    w = _gpu_quant(Wt)
+    packed, q, S = R.quantize(Wt)
+    assert np.array_equal(_np(w.codes), packed)
+    assert np.array_equal(_np(w.absmax_q), q)
+
+
 def test_quantize_absmax_debug_output():
     W = WL.weight(64, 1024, 0.02, seed=3)
     absmax = torch.empty(64 * 1024 // 64, dtype=torch.float32, device=DEV)
