@@ -190,9 +190,15 @@ int qlora_linear_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w, co
   if (m <= kSmallM) {
     if (lora) e = launch_lora_proj_small(X, m, w->k, A, r, scale, T, s);
     if (e == cudaSuccess) e = prof_mark(t_prof_start, s);
-    if (e == cudaSuccess)
-      e = launch_gemv_fwd(X, m, w->codes, w->absmax_q, w->group_scale, w->n, w->k, T, lora ? B : nullptr,
-                          lora ? r : 0, Y, s, pdl);
+    if (e == cudaSuccess) {
+      // Decode sizes take the per-warp streaming kernel; the rest (m > 4,
+      // or K beyond one cluster's warps) the CTA-ring kernel.
+      e = gemv_stream_supported(m, w->n, w->k)
+              ? launch_gemv_stream(X, m, w->codes, w->absmax_q, w->group_scale, w->n, w->k, T,
+                                   lora ? B : nullptr, lora ? r : 0, Y, s, pdl)
+              : launch_gemv_fwd(X, m, w->codes, w->absmax_q, w->group_scale, w->n, w->k, T, lora ? B : nullptr,
+                                lora ? r : 0, Y, s, pdl);
+    }
   } else {
     if (lora) e = tc_proj_kmajor(X, m, w->k, A, r, scale, T, s);
     if (e == cudaSuccess) e = prof_mark(t_prof_start, s);

@@ -92,6 +92,92 @@ __device__ __forceinline__ void decode8(uint32_t w, const Bf16Table &t, uint32_t
 }
 
 // ---------------------------------------------------------------------------
+// Thread-block clusters, distributed shared memory, warp-level MMA
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA of the cluster; orders shared-memory writes
+// before the barrier with distributed reads after it.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// fp32 at `local_addr` in the shared memory of cluster CTA `rank`.
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+// d += A(16x16, row) . B(16x8, col), bf16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// d = A(16x16, row) . B(16x8, col) with a zero accumulator.
+__device__ __forceinline__ void mma_bf16_16816_zero(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                    uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
+// Byte-pair table: entry b (two weights) holds {NF4[b >> 4], NF4[b & 15]} as a
+// bf16 pair, in 32 lane-private copies 256 bytes apart (entry b of lane l at
+// b * 256 + 4 l), so the 32 lookups of a warp always fall in 32 banks.
+constexpr uint32_t kPairLutBytes = 256u * 256u;
+
+__device__ __forceinline__ void build_pair_lut(uint8_t *lut, const Nf4Tables &tab, int tid, int nthreads) {
+  uint4 *lw = reinterpret_cast<uint4 *>(lut);
+  for (int i = tid; i < 256 * 16; i += nthreads) {
+    const int b = i >> 4;
+    const uint32_t v = pack_bf16x2(tab.level[b >> 4], tab.level[b & 15]);
+    lw[i] = make_uint4(v, v, v, v);
+  }
+}
+
+// Table offset of byte J (0..3) of `word` for the lane whose lane*4 is lane4.
+template <int J>
+__device__ __forceinline__ uint32_t pair_lut_off(uint32_t word, uint32_t lane4) {
+  return prmt(word, lane4, 0x5504u | (J << 4));
+}
+
+// Byte J of w as an exact float (0..255).
+template <int J>
+__device__ __forceinline__ float byte_to_f32(uint32_t w) {
+  return __uint_as_float(prmt(w, 0x4B000000u, 0x7650u | J)) - 8388608.0f;
+}
+
+// fp32(s / 255) correctly rounded: Markstein's division with the correctly
+// rounded reciprocal y = RN(1/255): q0 = RN(s y), the remainder
+// rho = s - 255 q0 is exact in one fma, and q0 + rho y rounds to the nearest
+// quotient.  IEEE division below 2^-100, where the remainder could lose bits.
+__device__ __forceinline__ float div255_rn(float s) {
+  if (!(s >= 0x1p-100f)) return __fdiv_rn(s, 255.0f);
+  const float y = 1.0f / 255.0f;
+  const float q0 = __fmul_rn(s, y);
+  const float rho = __fmaf_rn(-q0, 255.0f, s);
+  return __fmaf_rn(rho, y, q0);
+}
+
+// ---------------------------------------------------------------------------
 // mbarrier / fences / timers
 // ---------------------------------------------------------------------------
 

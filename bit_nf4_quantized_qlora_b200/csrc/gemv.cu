@@ -1,4 +1,6 @@
 // Small-M forward (M <= 16): Y = bf16(X . W^T + T . B^T), weight-streaming.
+// Decode sizes (M <= 4, K up to 32768) take the per-warp streaming kernel of
+// gemv_stream.cu; this CTA-ring kernel serves M = 5..16 and longer K.
 //
 // At decode-sized M the layer is bound by reading the packed weights from HBM
 // ("QLoRA and Quantized Training", The idea: dequantize each block, multiply,
@@ -34,7 +36,7 @@ constexpr int kStageBlocks = 4;                        // NF4 blocks of K per st
 constexpr uint32_t kStageBytes = kRows * kStageBlocks * 32u;   // 16 KB
 constexpr int kStages = 2;                             // x 2 CTAs per SM
 constexpr int kMaxM = 16;
-constexpr uint32_t kLutBytes = 256u * 256u;            // 256 entries x 256-byte stride
+constexpr uint32_t kLutBytes = kPairLutBytes;
 constexpr uint32_t kSmemBytes = kLutBytes + 1024u + kStages * kStageBytes + kMaxM * kRows * 4u;
 
 struct __align__(64) GemvParams {
@@ -51,34 +53,6 @@ struct __align__(64) GemvParams {
   Nf4Tables tab;
 };
 
-__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t cluster_size() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-  return v;
-}
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
@@ -89,12 +63,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
-}
-
-// LUT offset of byte j (0..3) of `word` for this lane: (byte << 8) | lane*4.
-template <int J>
-__device__ __forceinline__ uint32_t lut_off(uint32_t word, uint32_t lane4) {
-  return prmt(word, lane4, 0x5504u | (J << 4));
 }
 
 // One NF4 block (4 MMA k-steps) of this lane's two rows: returns the block's
@@ -110,28 +78,22 @@ __device__ __forceinline__ void block_mma(float (&bacc)[TOK_TILES][4], uint2 c0,
     const uint32_t w1 = ss < 2 ? c1.x : c1.y;
     uint32_t a[4];
     if ((ss & 1) == 0) {
-      a[0] = *reinterpret_cast<const uint32_t *>(lut + lut_off<0>(w0, lane4));
-      a[1] = *reinterpret_cast<const uint32_t *>(lut + lut_off<0>(w1, lane4));
-      a[2] = *reinterpret_cast<const uint32_t *>(lut + lut_off<1>(w0, lane4));
-      a[3] = *reinterpret_cast<const uint32_t *>(lut + lut_off<1>(w1, lane4));
+      a[0] = *reinterpret_cast<const uint32_t *>(lut + pair_lut_off<0>(w0, lane4));
+      a[1] = *reinterpret_cast<const uint32_t *>(lut + pair_lut_off<0>(w1, lane4));
+      a[2] = *reinterpret_cast<const uint32_t *>(lut + pair_lut_off<1>(w0, lane4));
+      a[3] = *reinterpret_cast<const uint32_t *>(lut + pair_lut_off<1>(w1, lane4));
     } else {
-      a[0] = *reinterpret_cast<const uint32_t *>(lut + lut_off<2>(w0, lane4));
-      a[1] = *reinterpret_cast<const uint32_t *>(lut + lut_off<2>(w1, lane4));
-      a[2] = *reinterpret_cast<const uint32_t *>(lut + lut_off<3>(w0, lane4));
-      a[3] = *reinterpret_cast<const uint32_t *>(lut + lut_off<3>(w1, lane4));
+      a[0] = *reinterpret_cast<const uint32_t *>(lut + pair_lut_off<2>(w0, lane4));
+      a[1] = *reinterpret_cast<const uint32_t *>(lut + pair_lut_off<2>(w1, lane4));
+      a[2] = *reinterpret_cast<const uint32_t *>(lut + pair_lut_off<3>(w0, lane4));
+      a[3] = *reinterpret_cast<const uint32_t *>(lut + pair_lut_off<3>(w1, lane4));
     }
 #pragma unroll
     for (int t = 0; t < TOK_TILES; ++t) {
       const uint4 &xv = ss < 2 ? xa[t] : xb[t];
-      mma_16816(bacc[t], a, (ss & 1) ? xv.z : xv.x, (ss & 1) ? xv.w : xv.y);
+      mma_bf16_16816(bacc[t], a[0], a[1], a[2], a[3], (ss & 1) ? xv.z : xv.x, (ss & 1) ? xv.w : xv.y);
     }
   }
-}
-
-// Absmax code byte j of a word -> float (exact for 0..255).
-template <int J>
-__device__ __forceinline__ float qbyte(uint32_t w) {
-  return __uint_as_float(prmt(w, 0x4B000000u, 0x7650u | J)) - 8388608.0f;
 }
 
 template <int TOK_TILES>
@@ -167,15 +129,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
     }
     fence_mbar_init();
   }
-  {
-    // Entry b (256 bytes): 32 copies of the pair, written 4 copies per store.
-    uint4 *lw = reinterpret_cast<uint4 *>(dsmem);
-    for (int i = threadIdx.x; i < 256 * 8; i += kThreads) {
-      const int b = i >> 3;
-      const uint32_t v = pack_bf16x2(p.tab.level[b >> 4], p.tab.level[b & 15]);
-      lw[b * 16 + (i & 7)] = make_uint4(v, v, v, v);
-    }
-  }
+  build_pair_lut(dsmem, p.tab, threadIdx.x, kThreads);
   __syncthreads();
 
   if (warp == kConsumers) {
@@ -246,8 +200,8 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
       if (full && qwords) {
         const uint32_t w0 = __ldg(reinterpret_cast<const uint32_t *>(q0p + st * kStageBlocks));
         const uint32_t w1 = __ldg(reinterpret_cast<const uint32_t *>(q1p + st * kStageBlocks));
-        qf0[0] = qbyte<0>(w0); qf0[1] = qbyte<1>(w0); qf0[2] = qbyte<2>(w0); qf0[3] = qbyte<3>(w0);
-        qf1[0] = qbyte<0>(w1); qf1[1] = qbyte<1>(w1); qf1[2] = qbyte<2>(w1); qf1[3] = qbyte<3>(w1);
+        qf0[0] = byte_to_f32<0>(w0); qf0[1] = byte_to_f32<1>(w0); qf0[2] = byte_to_f32<2>(w0); qf0[3] = byte_to_f32<3>(w0);
+        qf1[0] = byte_to_f32<0>(w1); qf1[1] = byte_to_f32<1>(w1); qf1[2] = byte_to_f32<2>(w1); qf1[3] = byte_to_f32<3>(w1);
       } else {
 #pragma unroll
         for (int b = 0; b < kStageBlocks; ++b) {

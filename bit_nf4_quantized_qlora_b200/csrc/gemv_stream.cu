@@ -1,0 +1,510 @@
+// Decode-sized forward (M <= 4): Y = bf16(X . W^T + T . B^T), streaming the
+// packed weights from HBM at close to copy bandwidth.
+//
+// At decode M the layer reads each packed weight once and does a couple of
+// FLOPs with it ("QLoRA and Quantized Training", The idea: dequantize each
+// block, multiply, discard), so the kernel is built around the load-store
+// unit, which every byte of codes passes through twice (once arriving, once
+// as a table lookup):
+//
+//   * Memory side.  A CTA owns a run of 16-row tiles; its 16 warps split K in
+//     chunks of 4 NF4 blocks (128 bytes of a row), so at any moment a CTA
+//     reads 16 rows x 2 KB of contiguous bytes.  Each warp streams its own
+//     chunk of successive tiles through a private 3-slot ring: one lane issues
+//     a TMA copy of the 16 x 128-byte box (plus the 16 x 16-byte box of absmax
+//     codes around it) on the slot's mbarrier.  No CTA-wide barriers, no
+//     producer warp; TMA writes bypass the load-store pipe, and the 128-byte
+//     swizzle with a row order that pairs rows r and r+4 in each quarter-warp
+//     makes the 16-byte reads conflict-free.
+//   * Expansion.  A 64 KB shared table maps every code byte (two weights) to
+//     the bf16 pair {NF4[hi], NF4[lo]} (32 lane-private copies, so lookups
+//     never conflict); the pairs are the A operand of m16n8k16 tensor-core
+//     MMAs whose B operand is X, kept in registers for the whole kernel.
+//   * Absmax scaling after the MMA.  A lane's 16 bytes are half of one NF4
+//     block, so the four lanes of an MMA row group cover two blocks.  The
+//     block is carried in the MMA's N dimension: column 2t holds token t on
+//     the lanes holding the first block of the pair, column 2t+1 token t on
+//     the lanes holding the second.  One MMA chain gives both blocks' raw sums
+//     side by side and each is scaled by its own c' = q * fp32(S/255) in fp32
+//     (fp32(S/255) is tabulated per group once per CTA, and applied once per
+//     row and chunk when the chunk lies in one group).  Columns are spare at
+//     M <= 4.
+//   * K split.  Chunks beyond one CTA's 16 warps go to the other CTAs of a
+//     thread-block cluster; warps add their per-tile partial sums into a
+//     shared buffer, the cluster reduces it through distributed shared memory,
+//     and the adapter term T . B^T is added before Y is written once in bf16.
+//     T comes from the preceding projection kernel, which this kernel
+//     overlaps (programmatic dependent launch) and waits for only before its
+//     epilogue.
+#include <cuda.h>
+
+#include <type_traits>
+#include <utility>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace qlora {
+namespace {
+
+constexpr int kWarps = 16;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kMaxM = 4;                 // two N columns per token in one n8 MMA
+constexpr int kMaxTiles = 64;            // 16-row tiles per CTA held in the reduction buffer
+constexpr int kMaxCluster = 8;
+constexpr int kMaxKBlocks = kMaxCluster * kWarps * 4;
+constexpr int kStages = 3;                // ring slots per warp (two in flight while one is read)
+constexpr uint32_t kCodeSlot = 16u * 128u;   // 16 rows x 4 blocks of codes
+constexpr uint32_t kQSlot = 16u * 16u;       // 16 rows x 16 absmax codes
+constexpr uint32_t kRedBytes = kMaxTiles * 16u * kMaxM * 4u;
+constexpr uint32_t kMaxGroups = (kMaxTiles * 16u * kMaxKBlocks) / 256u + 2u;
+constexpr uint32_t kTabBytes = (kMaxGroups * 4u + 1023u) & ~1023u;
+constexpr uint32_t kRingOff = kPairLutBytes + kRedBytes + kTabBytes;          // 1024-aligned
+constexpr uint32_t kQRingOff = kRingOff + kWarps * kStages * kCodeSlot;
+constexpr uint32_t kBarOff = kQRingOff + kWarps * kStages * kQSlot;
+constexpr uint32_t kSmemBytes = kBarOff + kWarps * kStages * 8u + 1024u;   // + base alignment slack
+static_assert(kRingOff % 1024u == 0, "128-byte swizzled boxes need 1024-byte alignment");
+static_assert(kSmemBytes <= 227u * 1024u, "shared memory");
+
+// MODE 2: k/64 % 16 == 0 (absmax codes by TMA, one group per chunk);
+// MODE 1: k/64 % 4 == 0 (absmax codes as words, one group per chunk);
+// MODE 0: any k/64 (byte loads, a group may change inside a chunk).
+struct __align__(64) StreamParams {
+  CUtensorMap tmCodes;           // codes [n x k/2] bytes, box {128, 16}, 128B swizzle
+  CUtensorMap tmQ;               // absmax codes [n x k/64] bytes, box {16, 16} (MODE 2)
+  const uint8_t *absmax_q;       // [n x k/64]
+  const float *group_scale;      // [ceil(n k / 16384)]
+  const uint16_t *X;             // [m x k] bf16
+  const uint16_t *T;             // [m x r] bf16 (adapter intermediate) or null
+  const uint16_t *B;             // [n x r] bf16
+  uint16_t *Y;                   // [m x n] bf16
+  unsigned *err;
+  int64_t n, k;
+  int m, r;
+  int ntiles;                    // ceil(n / 16)
+  int chunks;                    // ceil((k / 64) / 4)
+  int chunks_per_cta;            // chunks owned by one CTA of a cluster (<= 16)
+  Nf4Tables tab;
+};
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+// On lanes with `pred` set: expect `bytes` on the slot's mbarrier and start
+// the TMA copy of the codes box (and, if qmap is non-zero, of the absmax-code
+// box) into the slot.  Predicated rather than branched: every lane runs it.
+__device__ __forceinline__ void issue_unit(uint32_t pred, uint32_t bar, uint32_t bytes, uint32_t dst, uint64_t map,
+                                           int x, uint32_t qdst, uint64_t qmap, int qx, int y) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.u32 p, %0, 0;\n\t"
+      "@p fence.proxy.async.shared::cta;\n\t"
+      "@p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%1], %2;\n\t"
+      "@p cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%3], [%4, {%5, %9}], [%1];\n\t"
+      "}" ::"r"(pred), "r"(bar), "r"(bytes), "r"(dst), "l"(map), "r"(x), "r"(qdst), "l"(qmap), "r"(qx), "r"(y)
+      : "memory");
+  if (qmap != 0)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.u32 p, %0, 0;\n\t"
+        "@p cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%2], [%3, {%4, %5}], [%1];\n\t"
+        "}" ::"r"(pred), "r"(bar), "r"(qdst), "l"(qmap), "r"(qx), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t try_wait_u32(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok;
+}
+
+// Adds a and b at addr and addr + 32 bytes when pred is set.
+__device__ __forceinline__ void red_pair(uint32_t pred, uint32_t addr, float a, float b) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.u32 p, %0, 0;\n\t"
+      "@p red.shared.add.f32 [%1], %2;\n\t"
+      "@p red.shared.add.f32 [%1+32], %3;\n\t}" ::"r"(pred), "r"(addr), "f"(a), "f"(b)
+      : "memory");
+}
+
+// Two k-steps from one 32-bit word of each of the rows g and g+8 (8 weights
+// each): byte 0 -> a0/a1, byte 1 -> a2/a3, then bytes 2 and 3.  xv holds the
+// matching 8 activations of this lane's column.  FIRST starts the chain from
+// a zero accumulator.
+template <bool FIRST>
+__device__ __forceinline__ void word_mma(float (&d)[4], uint32_t w_g, uint32_t w_g8, const uint8_t *lut, uint32_t lane4,
+                                         const uint4 &xv) {
+  const auto L = [&](uint32_t off) { return *reinterpret_cast<const uint32_t *>(lut + off); };
+  const uint32_t a0 = L(pair_lut_off<0>(w_g, lane4)), a1 = L(pair_lut_off<0>(w_g8, lane4));
+  const uint32_t a2 = L(pair_lut_off<1>(w_g, lane4)), a3 = L(pair_lut_off<1>(w_g8, lane4));
+  if (FIRST)
+    mma_bf16_16816_zero(d, a0, a1, a2, a3, xv.x, xv.y);
+  else
+    mma_bf16_16816(d, a0, a1, a2, a3, xv.x, xv.y);
+  mma_bf16_16816(d, L(pair_lut_off<2>(w_g, lane4)), L(pair_lut_off<2>(w_g8, lane4)), L(pair_lut_off<3>(w_g, lane4)),
+                 L(pair_lut_off<3>(w_g8, lane4)), xv.z, xv.w);
+}
+
+template <class F, int... S>
+__device__ __forceinline__ bool slot_pass(const F &f, uint32_t ph, std::integer_sequence<int, S...>) {
+  return f(ph, std::integral_constant<int, S>{}...);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_constant__ StreamParams p) {
+  extern __shared__ __align__(1024) uint8_t dsmem[];
+  const uint8_t *lut = dsmem;
+  float *red = reinterpret_cast<float *>(dsmem + kPairLutBytes);
+  float *ttab = reinterpret_cast<float *>(dsmem + kPairLutBytes + kRedBytes);
+  // Ring offsets are taken from a 1024-aligned base (the 128-byte swizzle
+  // pattern is defined on 1024-byte atoms of shared memory).
+  const uint32_t sbase = smem_u32(dsmem);
+  const uint32_t abase = (sbase + 1023u) & ~1023u;
+  const uint32_t ring = abase + kRingOff;
+  const uint32_t qring = abase + kQRingOff;
+  const uint32_t bars = abase + kBarOff;
+
+  const uint32_t crank = cluster_rank();
+  const uint32_t csize = cluster_size();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, q = lane & 3;
+  const int ncl = static_cast<int>(gridDim.y);
+  const int cl = static_cast<int>(blockIdx.y);
+  const int t_lo = static_cast<int>((static_cast<int64_t>(p.ntiles) * cl) / ncl);
+  const int t_hi = static_cast<int>((static_cast<int64_t>(p.ntiles) * (cl + 1)) / ncl);
+  const int nt = t_hi - t_lo;
+  const int kblocks = static_cast<int>(p.k >> 6);
+
+  // Warp -> (chunk, tile phase): with fewer chunks than warps, several warps
+  // take the same chunk on interleaved tiles.
+  const int cpc = p.chunks_per_cta;
+  const int phases = kWarps / cpc;
+  const int phase = warp / cpc;
+  const int chunk = static_cast<int>(crank) * cpc + warp % cpc;
+  const bool active = phase < phases && chunk < p.chunks;
+  const int kb0 = chunk * 4;
+  const int nvalid = min(4, kblocks - kb0);
+  const int nunits = active && nt > phase ? (nt - phase + phases - 1) / phases : 0;
+  const uint32_t tx_bytes = kCodeSlot + (MODE == 2 ? kQSlot : 0u);
+  const uint64_t map_codes = reinterpret_cast<uint64_t>(&p.tmCodes);
+  const uint64_t map_q = MODE == 2 ? reinterpret_cast<uint64_t>(&p.tmQ) : 0ull;
+  const uint32_t bar_w = bars + warp * kStages * 8u;                     // slot s: + 8 s
+  const uint32_t ring_w = ring + warp * kStages * kCodeSlot;              // slot s: + s kCodeSlot
+  const uint32_t qring_w = qring + warp * kStages * kQSlot;               // slot s: + s kQSlot
+  const int y_step = 16 * phases;
+  // Each warp's ring starts filling before the tables are built.
+  if (lane == 0) {
+    for (int s = 0; s < kStages; ++s)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_w + s * 8u));
+    fence_mbar_init();
+  }
+  __syncwarp();
+  for (int s = 0; s < kStages && s < nunits; ++s)
+    issue_unit(lane == 0, bar_w + s * 8u, tx_bytes, ring_w + s * kCodeSlot, map_codes, kb0 * 32,
+               qring_w + s * kQSlot, map_q, kb0 & ~15, (t_lo + phase) * 16 + s * y_step);
+
+  // fp32(S / 255) of every group the CTA's rows touch.  Rows of the last
+  // tile past n (codes and absmax codes read as zero) index the table too;
+  // their entries repeat the last group.  Row * k/64 fits in 32 bits
+  // (checked on the host).
+  const int gbase = (t_lo * 16 * kblocks) >> 8;
+  const int ngroups = ((t_hi * 16 * kblocks - 1) >> 8) - gbase + 1;
+  const int glast = static_cast<int>((p.n * kblocks - 1) >> 8);
+  for (int i = threadIdx.x; i < ngroups; i += kThreads)
+    ttab[i] = div255_rn(__ldg(p.group_scale + min(gbase + i, glast)));
+  build_pair_lut(dsmem, p.tab, threadIdx.x, kThreads);
+  for (int i = threadIdx.x; i < nt * 16 * kMaxM; i += kThreads) red[i] = 0.f;
+
+  // B operand (X): column g = 2 * token + block parity; lanes whose piece is
+  // in the other block of the pair, and tokens >= m, hold zeros.
+  const int tok = g >> 1;
+  const bool live = active && (g & 1) == (q >> 1) && tok < p.m;
+  uint4 xf[2][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool v = live && (MODE != 0 || 2 * i + (q >> 1) < nvalid);
+    const uint4 *xp = reinterpret_cast<const uint4 *>(p.X + static_cast<int64_t>(v ? tok : 0) * p.k +
+                                                      (v ? kb0 * 64 + 64 * (2 * i + (q >> 1)) + 32 * (q & 1) : 0));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) xf[i][j] = v ? __ldg(xp + j) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  __syncthreads();
+
+  if (active) {
+    const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
+    // MMA row group g reads physical rows pr and pr + 8 of the tile, with pr
+    // pairing rows r and r + 4 in each quarter-warp: the two rows' swizzle
+    // phases then differ in the chunk index's top bit.
+    const int pr = (g >> 1) + 4 * (g & 1);
+    const uint32_t off_r0_p0 = static_cast<uint32_t>(pr) * 128u + ((static_cast<uint32_t>(q) ^ pr) << 4);
+    const uint32_t off_r0_p1 = static_cast<uint32_t>(pr) * 128u + ((static_cast<uint32_t>(4 + q) ^ pr) << 4);
+    const uint32_t off_r1_p0 = off_r0_p0 + 8u * 128u;
+    const uint32_t off_r1_p1 = off_r0_p1 + 8u * 128u;
+
+    const uint32_t tab_w = smem_u32(ttab) - 4u * static_cast<uint32_t>(gbase);
+    const uint32_t qoff0 = static_cast<uint32_t>(pr) * 16u + (kb0 & 15), qoff1 = qoff0 + 8u * 16u;
+    const uint32_t red_pred = q < p.m ? 1u : 0u;
+    // Loop state: rk = row * k/64 + kb0 for the rows pr and pr + 8 of the
+    // current tile; y_refill is the first row of the unit kStages ahead.
+    int rk0 = ((t_lo + phase) * 16 + pr) * kblocks + kb0;
+    const int rk_step = 16 * phases * kblocks, rk_8 = 8 * kblocks;
+    int y_refill = (t_lo + phase) * 16 + kStages * y_step;
+    const int y_end = t_hi * 16;
+    uint32_t red_addr = smem_u32(red) + 4u * static_cast<uint32_t>((phase * kMaxM + q) * 16 + pr);
+    const uint32_t red_step = 4u * static_cast<uint32_t>(phases * kMaxM * 16);
+    const int nm1 = static_cast<int>(p.n) - 1;
+    int u = phase;
+
+    // One unit (this warp's chunk of one tile) from ring slot S; false when
+    // the warp is done or a wait gave up.
+    const auto unit = [&](auto s_const, uint32_t ph) -> bool {
+      constexpr int S = decltype(s_const)::value;
+      if (u >= nt) return false;
+      const int rk1 = rk0 + rk_8;
+      uint32_t qw0 = 0, qw1 = 0;
+      float tlo0 = __uint_as_float(lds32(tab_w + 4u * static_cast<uint32_t>(rk0 >> 8)));
+      float tlo1 = __uint_as_float(lds32(tab_w + 4u * static_cast<uint32_t>(rk1 >> 8)));
+      float thi0 = tlo0, thi1 = tlo1;
+      int split0 = 4, split1 = 4;   // blocks of the chunk before each row's next group
+      if (MODE != 2) {
+        // Absmax codes by plain loads, from rows clamped to the matrix.
+        const int tile_row = (t_lo + u) * 16;
+        const int64_t bq0 = static_cast<int64_t>(min(tile_row + pr, nm1)) * kblocks + kb0;
+        const int64_t bq1 = static_cast<int64_t>(min(tile_row + pr + 8, nm1)) * kblocks + kb0;
+        if (MODE == 1) {
+          qw0 = __ldg(reinterpret_cast<const uint32_t *>(p.absmax_q + bq0));
+          qw1 = __ldg(reinterpret_cast<const uint32_t *>(p.absmax_q + bq1));
+        } else {
+          for (int b = 0; b < nvalid; ++b) {
+            qw0 |= static_cast<uint32_t>(__ldg(p.absmax_q + bq0 + b)) << (8 * b);
+            qw1 |= static_cast<uint32_t>(__ldg(p.absmax_q + bq1 + b)) << (8 * b);
+          }
+          thi0 = __uint_as_float(lds32(tab_w + 4u * static_cast<uint32_t>((rk0 + nvalid - 1) >> 8)));
+          thi1 = __uint_as_float(lds32(tab_w + 4u * static_cast<uint32_t>((rk1 + nvalid - 1) >> 8)));
+          split0 = 256 - (rk0 & 255);
+          split1 = 256 - (rk1 & 255);
+        }
+      }
+      // A wait that gives up (it never should) ends the warp's loop on every
+      // lane together.
+      const uint32_t bar = bar_w + S * 8u;
+      if (__any_sync(0xffffffffu, try_wait_u32(bar, ph) == 0u)) {
+        uint64_t *barp = reinterpret_cast<uint64_t *>(dsmem + (bar - sbase));
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(barp, ph, p.err, kErrTimeoutFullA))) return false;
+      }
+      const uint32_t slot = ring_w + S * kCodeSlot;
+      const uint4 c00 = lds128(slot + off_r0_p0), c01 = lds128(slot + off_r0_p1);
+      const uint4 c10 = lds128(slot + off_r1_p0), c11 = lds128(slot + off_r1_p1);
+      if (MODE == 2) {
+        qw0 = lds32(qring_w + S * kQSlot + qoff0);
+        qw1 = lds32(qring_w + S * kQSlot + qoff1);
+      }
+      float acc0, acc1;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        float d[4];
+        const uint4 cg = i == 0 ? c00 : c01, cg8 = i == 0 ? c10 : c11;
+        word_mma<true>(d, cg.x, cg8.x, lut, lane4, xf[i][0]);
+        word_mma<false>(d, cg.y, cg8.y, lut, lane4, xf[i][1]);
+        word_mma<false>(d, cg.z, cg8.z, lut, lane4, xf[i][2]);
+        word_mma<false>(d, cg.w, cg8.w, lut, lane4, xf[i][3]);
+        // d[0], d[1]: row pr, token q, blocks 2i and 2i+1; d[2], d[3]: row pr + 8.
+        const float qa0 = i == 0 ? byte_to_f32<0>(qw0) : byte_to_f32<2>(qw0);
+        const float qb0 = i == 0 ? byte_to_f32<1>(qw0) : byte_to_f32<3>(qw0);
+        const float qa1 = i == 0 ? byte_to_f32<0>(qw1) : byte_to_f32<2>(qw1);
+        const float qb1 = i == 0 ? byte_to_f32<1>(qw1) : byte_to_f32<3>(qw1);
+        if (MODE != 0) {
+          // One group per chunk: fp32(S/255) is common to the four blocks
+          // and is applied once per row below.
+          acc0 = i == 0 ? qa0 * d[0] : fmaf(qa0, d[0], acc0);
+          acc1 = i == 0 ? qa1 * d[2] : fmaf(qa1, d[2], acc1);
+          acc0 = fmaf(qb0, d[1], acc0);
+          acc1 = fmaf(qb1, d[3], acc1);
+        } else {
+          const float ta0 = 2 * i < split0 ? tlo0 : thi0, tb0 = 2 * i + 1 < split0 ? tlo0 : thi0;
+          const float ta1 = 2 * i < split1 ? tlo1 : thi1, tb1 = 2 * i + 1 < split1 ? tlo1 : thi1;
+          acc0 = i == 0 ? __fmul_rn(qa0, ta0) * d[0] : fmaf(__fmul_rn(qa0, ta0), d[0], acc0);
+          acc1 = i == 0 ? __fmul_rn(qa1, ta1) * d[2] : fmaf(__fmul_rn(qa1, ta1), d[2], acc1);
+          acc0 = fmaf(__fmul_rn(qb0, tb0), d[1], acc0);
+          acc1 = fmaf(__fmul_rn(qb1, tb1), d[3], acc1);
+        }
+      }
+      if (MODE != 0) {
+        acc0 *= tlo0;
+        acc1 *= tlo1;
+      }
+      // The slot's bytes are consumed: refill it with the unit kStages ahead.
+      __syncwarp();
+      issue_unit(lane == 0 && y_refill < y_end, bar, tx_bytes, slot, map_codes, kb0 * 32, qring_w + S * kQSlot,
+                 map_q, kb0 & ~15, y_refill);
+      red_pair(red_pred, red_addr, acc0, acc1);
+      y_refill += y_step;
+      red_addr += red_step;
+      rk0 += rk_step;
+      u += phases;
+      return true;
+    };
+
+    // The ring is walked slot by slot with compile-time slot indices; the
+    // mbarrier phase flips after every pass over the ring.
+    int j = 0;
+    const auto pass = [&](uint32_t ph, auto... s) { return ((unit(s, ph) && (++j, true)) && ...); };
+    for (uint32_t ph = 0;; ph ^= 1u)
+      if (!slot_pass(pass, ph, std::make_integer_sequence<int, kStages>{})) break;
+    const bool ok = u >= nt;
+    if (!ok && lane == 0) {
+      // A wait gave up: let copies still in flight land before the CTA's
+      // memory is released.
+      for (int jj = j; jj < j + kStages && jj < nunits; ++jj) {
+        uint64_t *b = reinterpret_cast<uint64_t *>(dsmem + (bar_w - sbase) + (jj % kStages) * 8u);
+        mbar_wait_bounded(b, static_cast<uint32_t>(jj / kStages) & 1u, p.err, kErrTimeoutDrain);
+      }
+    }
+  }
+  __syncthreads();
+  cluster_sync_all();
+
+  // The adapter intermediate T is written by the preceding kernel (a no-op
+  // when this grid was not launched as its programmatic dependent).
+  if (p.r > 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+  // CTA `crank` finishes its share of the cluster's (tile, token, row) sums.
+  const int total = nt * p.m * 16;
+  const int o_lo = static_cast<int>((static_cast<int64_t>(total) * crank) / csize);
+  const int o_hi = static_cast<int>((static_cast<int64_t>(total) * (crank + 1)) / csize);
+  const uint32_t red_addr = smem_u32(red);
+  for (int o = o_lo + static_cast<int>(threadIdx.x); o < o_hi; o += kThreads) {
+    const int ut = o / (p.m * 16);
+    const int rem = o - ut * p.m * 16;
+    const int mi = rem >> 4, rl = rem & 15;
+    const int64_t n = static_cast<int64_t>(t_lo + ut) * 16 + rl;
+    if (n >= p.n) continue;
+    const uint32_t off = red_addr + static_cast<uint32_t>((ut * kMaxM + mi) * 16 + rl) * 4u;
+    float sum = 0.f;
+    for (uint32_t peer = 0; peer < csize; ++peer) sum += ld_dsmem_f32(off, peer);
+    if (p.r > 0) {
+      const uint16_t *trow = p.T + static_cast<int64_t>(mi) * p.r;
+      const uint16_t *brow = p.B + n * p.r;
+      for (int jr = 0; jr < p.r; jr += 8) {
+        const uint4 tv = *reinterpret_cast<const uint4 *>(trow + jr);
+        const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(brow + jr));
+        const uint32_t ta[4] = {tv.x, tv.y, tv.z, tv.w};
+        const uint32_t ba[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          sum = fmaf(bf16lo_to_f32(ta[e]), bf16lo_to_f32(ba[e]), sum);
+          sum = fmaf(bf16hi_to_f32(ta[e]), bf16hi_to_f32(ba[e]), sum);
+        }
+      }
+    }
+    p.Y[static_cast<int64_t>(mi) * p.n + n] = static_cast<uint16_t>(pack_bf16x2(sum, 0.f) & 0xFFFFu);
+  }
+  cluster_sync_all();
+}
+
+template <int MODE>
+cudaError_t configure(int dev) {
+  static bool done[64] = {};
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (done[dev]) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(gemv_stream_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kSmemBytes));
+  if (e == cudaSuccess) done[dev] = true;
+  return e;
+}
+
+template <int MODE>
+cudaError_t launch_mode(const StreamParams &p, int dev, int sms, int cs, cudaStream_t stream, bool pdl) {
+  cudaError_t e = configure<MODE>(dev);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(cs), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(cs);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // One CTA per SM: as many clusters as can be resident at once (the GPC
+  // layout may hold fewer than sms / cs), each with a contiguous run of at
+  // most kMaxTiles tiles.
+  static int resident[64][kMaxCluster + 1] = {};
+  int &res = resident[dev][cs];
+  if (res == 0) {
+    int v = 0;
+    e = cudaOccupancyMaxActiveClusters(&v, gemv_stream_kernel<MODE>, &cfg);
+    if (e != cudaSuccess) return e;
+    res = v > 0 ? v : (sms / cs > 0 ? sms / cs : 1);
+  }
+  int ncl = res < p.ntiles ? res : p.ntiles;
+  const int min_ncl = (p.ntiles + kMaxTiles - 1) / kMaxTiles;
+  if (ncl < min_ncl) ncl = min_ncl;
+  cfg.gridDim = dim3(static_cast<unsigned>(cs), static_cast<unsigned>(ncl), 1);
+  cfg.numAttrs = (p.r > 0 && pdl) ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, gemv_stream_kernel<MODE>, p);
+}
+
+}  // namespace
+
+bool gemv_stream_supported(int64_t m, int64_t n, int64_t k) {
+  // Row * k/64 indices (rows padded to whole tiles) are kept in 32 bits.
+  return m >= 1 && m <= kMaxM && k / 64 <= kMaxKBlocks && (n + 16) * (k / 64) < (int64_t(1) << 31);
+}
+
+cudaError_t launch_gemv_stream(const uint16_t *X, int64_t m, const uint8_t *codes, const uint8_t *absmax_q,
+                               const float *group_scale, int64_t n, int64_t k, const uint16_t *T,
+                               const uint16_t *B, int32_t r, uint16_t *Y, cudaStream_t stream, bool pdl) {
+  if (m <= 0) return cudaSuccess;
+  if (!gemv_stream_supported(m, n, k)) return cudaErrorInvalidValue;
+  const int64_t kblocks = k / 64;
+  const int mode = kblocks % 16 == 0 ? 2 : (kblocks % 4 == 0 ? 1 : 0);
+  StreamParams p{};
+  if (!encode_codes_map(&p.tmCodes, codes, n, k / 2, 128, 16, true)) return cudaErrorInvalidValue;
+  if (mode == 2 && !encode_codes_map(&p.tmQ, absmax_q, n, kblocks, 16, 16, false)) return cudaErrorInvalidValue;
+  p.absmax_q = absmax_q;
+  p.group_scale = group_scale;
+  p.X = X;
+  p.T = T;
+  p.B = B;
+  p.Y = Y;
+  p.err = device_error_word();
+  p.n = n;
+  p.k = k;
+  p.m = static_cast<int>(m);
+  p.r = (T != nullptr && B != nullptr) ? r : 0;
+  p.ntiles = static_cast<int>((n + 15) / 16);
+  p.chunks = static_cast<int>((kblocks + 3) / 4);
+  const int cs = (p.chunks + kWarps - 1) / kWarps;
+  p.chunks_per_cta = (p.chunks + cs - 1) / cs;
+  p.tab = nf4_tables();
+
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const cudaError_t e = mode == 2   ? launch_mode<2>(p, dev, sms, cs, stream, pdl)
+                        : mode == 1 ? launch_mode<1>(p, dev, sms, cs, stream, pdl)
+                                    : launch_mode<0>(p, dev, sms, cs, stream, pdl);
+  if (e == cudaSuccess) count_launches(1);
+  return e;
+}
+
+}  // namespace qlora

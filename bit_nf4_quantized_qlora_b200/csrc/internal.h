@@ -42,12 +42,20 @@ cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *absmax_q, const 
 cudaError_t launch_lora_proj_small(const uint16_t *X, int64_t m, int64_t k, const uint16_t *A,
                                    int32_t r, float scale, uint16_t *T, cudaStream_t stream);
 
-// Y[m x n] = bf16(X . W^T + T . B^T) for m <= 16 (weight-streaming kernel);
-// with pdl it overlaps the preceding T projection.
+// Y[m x n] = bf16(X . W^T + T . B^T) for m <= 16 (CTA-ring weight-streaming
+// kernel); with pdl it overlaps the preceding T projection.
 cudaError_t launch_gemv_fwd(const uint16_t *X, int64_t m, const uint8_t *codes,
                             const uint8_t *absmax_q, const float *group_scale, int64_t n, int64_t k,
                             const uint16_t *T, const uint16_t *B, int32_t r, uint16_t *Y,
                             cudaStream_t stream, bool pdl);
+
+// Decode-sized forward (m <= 4, k/64 <= 512): per-warp TMA streams of the
+// codes, K split over a cluster.  Same contract as launch_gemv_fwd.
+bool gemv_stream_supported(int64_t m, int64_t n, int64_t k);
+cudaError_t launch_gemv_stream(const uint16_t *X, int64_t m, const uint8_t *codes,
+                               const uint8_t *absmax_q, const float *group_scale, int64_t n, int64_t k,
+                               const uint16_t *T, const uint16_t *B, int32_t r, uint16_t *Y,
+                               cudaStream_t stream, bool pdl);
 
 // tcgen05 paths -------------------------------------------------------------
 

@@ -167,27 +167,6 @@ struct Cfg {
   static_assert(!SPLIT || STAGE_BYTES * STAGES >= 128u * 64u * 4u, "room for the fp32 partial tile");
 };
 
-__device__ __forceinline__ uint32_t cl_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t cl_size() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cl_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ float ld_peer_f32(uint32_t local_addr, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-  return v;
-}
-
 template <class C>
 __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t dsmem[];
@@ -495,15 +474,15 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
   if (C::SPLIT) {
     // Reduce the cluster's partial tiles through distributed shared memory:
     // CTA `rank` finishes rows [rank*128/size, (rank+1)*128/size).
-    cl_sync();
-    const uint32_t rank = cl_rank(), size = cl_size();
+    cluster_sync_all();
+    const uint32_t rank = cluster_rank(), size = cluster_size();
     const int r_lo = static_cast<int>((128u * rank) / size), r_hi = static_cast<int>((128u * (rank + 1)) / size);
     const int rows = r_hi - r_lo;
     for (int i = threadIdx.x; i < rows * C::BN; i += C::NUM_THREADS) {
       const int col = i / rows, row = r_lo + (i % rows);
       const uint32_t off = base + (static_cast<uint32_t>(col) * 128u + static_cast<uint32_t>(row)) * 4u;
       float acc = 0.f;
-      for (uint32_t pr = 0; pr < size; ++pr) acc += ld_peer_f32(off, pr);
+      for (uint32_t pr = 0; pr < size; ++pr) acc += ld_dsmem_f32(off, pr);
       const int64_t grow = static_cast<int64_t>(m_tile) * C::BM + row;
       const int64_t gcol = static_cast<int64_t>(n_tile) * C::BN + col;
       if (grow < p.out_rows && gcol < p.out_cols) {
@@ -512,7 +491,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
         else p.out[grow * p.out_ld + gcol] = v;
       }
     }
-    cl_sync();
+    cluster_sync_all();
   }
   tc_fence_before();
   __syncthreads();

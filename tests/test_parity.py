@@ -137,8 +137,11 @@ def test_dequant_bit_exact(shape):
 # ---------------------------------------------------------------------------
 
 FWD_CASES = [
-    # weight-streaming path (m <= 16)
+    # weight-streaming paths (m <= 16); m <= 4 takes the direct-load kernel: K ragged in chunks of
+    # four blocks, groups changing inside a chunk, n % 16 == 8, clusters of 3, 5 and 8 CTAs, and
+    # one K beyond a cluster's warps (back on the TMA-ring kernel)
     (1024, 1024, 16, 16), (1024, 1024, 1, 16), (72, 320, 3, 16), (264, 1088, 7, 0), (4096, 1024, 16, 64),
+    (264, 1088, 4, 0), (1032, 8256, 2, 32), (136, 16448, 1, 16), (24, 32768, 4, 16), (16, 33024, 1, 16),
     # tcgen05 path: several tiles plus ragged tails in m and n, k a few k-steps
     (520, 640, 200, 16), (264, 192, 17, 0), (1024, 1024, 300, 64), (256, 64, 130, 32), (776, 512, 129, 16),
 ]
