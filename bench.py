@@ -312,6 +312,84 @@ def _m1_decode(dev, peaks, peak_kind):
     return out
 
 
+def _decoder_layer(dev, steps: int = 5, warmup: int = 2):
+    """7B-shaped decoder block (q, k, v, o, gate, up, down all NF4 + LoRA
+    r=64, attention/RMSNorm/SwiGLU in PyTorch), X [2 x 2048 x 4096]: device
+    time of one forward + backward, and the seven projections' algorithmic
+    FLOPs over it."""
+    import torch
+    from bit_nf4_quantized_qlora_b200 import layer as L
+    from bit_nf4_quantized_qlora_b200 import workloads as WL
+    case = WL.DecoderLayerCase()
+    block = L.build_decoder(case, dev)
+    x = case.X().to(dev).requires_grad_(True)
+    gy = case.grad().to(dev)
+
+    def step():
+        for prm in block.parameters():
+            prm.grad = None
+        x.grad = None
+        block(x).backward(gy)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    t = t0.elapsed_time(t1) * 1e-3 / steps
+    fl = L.linear_flops(case, case.batch * case.seq)
+    del block, x, gy
+    torch.cuda.empty_cache()
+    return {"ms_per_step": round(t * 1e3, 3), "linear_tflops": round(fl["total"] / t / 1e12, 1),
+            "linear_flops_per_step": fl["total"], "steps": steps,
+            "shape": "hidden 4096, 32 heads x 128, MLP 11008, X [2 x 2048 x 4096], LoRA r=64 alpha=16",
+            "note": "FLOPs count the seven quantized projections (fwd, dX, adapter grads); attention, "
+                    "RMSNorm and SwiGLU run in PyTorch inside the timed step"}
+
+
+def _unfused_comparator(p, dev, reps: int = 10):
+    """The forward of one 7B MLP projection done the unfused way -- the
+    library's standalone dequant to a bf16 weight in HBM, then torch.matmul
+    (cuBLAS) for X W^T and the adapter products -- against the fused kernel
+    on the same inputs."""
+    import torch
+    from bit_nf4_quantized_qlora_b200 import binding as B
+    c = p.case
+    Wd = torch.empty(c.n, c.k, dtype=torch.bfloat16, device=dev)
+    Y = torch.empty(c.m, c.n, dtype=torch.bfloat16, device=dev)
+
+    def unfused():
+        B.qlora_dequant(p.w, out=Wd)
+        T = (p.X @ p.A.t()) * c.scale
+        torch.matmul(p.X, Wd.t(), out=Y)
+        Y.addmm_(T, p.B.t())
+
+    def fused():
+        B.qlora_linear_fwd(p.X, p.w, p.A, p.B, c.r, c.scale, out=Y, ws=p.ws_f)
+
+    out = {}
+    for name, fn in (("unfused_dequant_plus_cublas", unfused), ("fused", fused)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(reps):
+            fn()
+        t1.record()
+        torch.cuda.synchronize()
+        t = t0.elapsed_time(t1) * 1e-3 / reps
+        out[name] = {"us": round(t * 1e6, 1),
+                     "tflops": round(linear_flops(c.m, c.n, c.k, c.r)["fwd"] / t / 1e12, 1)}
+    out["workload"] = f"forward {c.m}x{c.n}x{c.k}, LoRA r={c.r} (7B MLP gate)"
+    del Wd
+    return out
+
+
 def _cpu_baseline(rank: int, world: int):
     if rank != 0 or world != 1:
         return None
@@ -395,6 +473,8 @@ def run_ours(args):
     e2e = _e2e(projs, cases, flat, world, dev, stream, max(3, min(K, 10)))
 
     m1 = _m1_decode(dev, peaks, peak_kind) if rank == 0 else None
+    layer = _decoder_layer(dev) if rank == 0 else None
+    unfused = _unfused_comparator(projs[0], dev) if rank == 0 else None
     cpu = _cpu_baseline(rank, world)
 
     if rank == 0:
@@ -413,6 +493,8 @@ def run_ours(args):
             "gpu_launches": int(launches),
             "clocks": clk.summary(),
             "m1_decode": m1,
+            "decoder_layer_7b": layer,
+            "unfused_comparator": unfused,
             "device_error_flags": dev_err,
         }
         print(json.dumps(line))

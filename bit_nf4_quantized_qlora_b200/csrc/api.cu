@@ -37,10 +37,21 @@ int cuda_status(cudaError_t e) {
 
 size_t round_up(size_t v) { return (v + kWsAlign - 1) / kWsAlign * kWsAlign; }
 
+// The device the calls run on must be sm_100.  The first call on a host
+// thread also makes sure the runtime has a context current on that thread
+// (a thread that never touched CUDA, such as a framework's worker thread, may
+// have none yet; kernel configuration calls made before it is bound have
+// failed with cudaErrorInvalidValue).
 int check_device() {
+  thread_local int t_ready_dev = -1;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_status(e);
+  if (t_ready_dev != dev) {
+    e = cudaFree(nullptr);
+    if (e != cudaSuccess) return cuda_status(e);
+    t_ready_dev = dev;
+  }
   int major = 0;
   e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
   if (e != cudaSuccess) return cuda_status(e);

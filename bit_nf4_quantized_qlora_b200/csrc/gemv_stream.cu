@@ -180,7 +180,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
 
   const uint32_t crank = cluster_rank();
   const uint32_t csize = cluster_size();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // The warp index read through a shuffle is known to be warp-uniform, so
+  // everything derived from it (ring, barrier and TMA operands) can live in
+  // uniform registers.
+  const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x >> 5), 0);
+  const int lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3;
   const int ncl = static_cast<int>(gridDim.y);
   const int cl = static_cast<int>(blockIdx.y);

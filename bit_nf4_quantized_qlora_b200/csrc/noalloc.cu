@@ -38,6 +38,8 @@ cudaError_t scratch_address(void **out) {
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
   if (g_scratch_ptr[dev] == nullptr) {
     void *p = nullptr;
+    e = cudaFree(nullptr);   // a context current on this thread before the lookup
+    if (e != cudaSuccess) return e;
     e = cudaGetSymbolAddress(&p, g_fwd_scratch);
     if (e != cudaSuccess) return e;
     g_scratch_ptr[dev] = p;
