@@ -50,14 +50,16 @@ namespace {
 constexpr int kWarps = 16;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kMaxM = 4;                 // two N columns per token in one n8 MMA
-constexpr int kMaxTiles = 64;            // 16-row tiles per CTA held in the reduction buffer
+constexpr int kTileRows = 32;            // weight rows per tile: two m16n8k16 row tiles
+constexpr int kSub = kTileRows / 16;
+constexpr int kMaxTiles = 16;            // tiles per CTA held in the reduction buffer
 constexpr int kMaxCluster = 8;
 constexpr int kMaxKBlocks = kMaxCluster * kWarps * 4;
-constexpr int kStages = 3;                // ring slots per warp (two in flight while one is read)
-constexpr uint32_t kCodeSlot = 16u * 128u;   // 16 rows x 4 blocks of codes
-constexpr uint32_t kQSlot = 16u * 16u;       // 16 rows x 16 absmax codes
-constexpr uint32_t kRedBytes = kMaxTiles * 16u * kMaxM * 4u;
-constexpr uint32_t kMaxGroups = (kMaxTiles * 16u * kMaxKBlocks) / 256u + 2u;
+constexpr int kStages = 2;                // ring slots per warp (one in flight while one is read)
+constexpr uint32_t kCodeSlot = kTileRows * 128u;   // tile rows x 4 blocks of codes
+constexpr uint32_t kQSlot = kTileRows * 16u;       // tile rows x 16 absmax codes
+constexpr uint32_t kRedBytes = kMaxTiles * kTileRows * kMaxM * 4u;
+constexpr uint32_t kMaxGroups = (kMaxTiles * kTileRows * kMaxKBlocks) / 256u + 2u;
 constexpr uint32_t kTabBytes = (kMaxGroups * 4u + 1023u) & ~1023u;
 constexpr uint32_t kRingOff = kPairLutBytes + kRedBytes + kTabBytes;          // 1024-aligned
 constexpr uint32_t kQRingOff = kRingOff + kWarps * kStages * kCodeSlot;
@@ -70,8 +72,8 @@ static_assert(kSmemBytes <= 227u * 1024u, "shared memory");
 // MODE 1: k/64 % 4 == 0 (absmax codes as words, one group per chunk);
 // MODE 0: any k/64 (byte loads, a group may change inside a chunk).
 struct __align__(64) StreamParams {
-  CUtensorMap tmCodes;           // codes [n x k/2] bytes, box {128, 16}, 128B swizzle
-  CUtensorMap tmQ;               // absmax codes [n x k/64] bytes, box {16, 16} (MODE 2)
+  CUtensorMap tmCodes;           // codes [n x k/2] bytes, box {128, tile rows}, 128B swizzle
+  CUtensorMap tmQ;               // absmax codes [n x k/64] bytes, box {16, tile rows} (MODE 2)
   const uint8_t *absmax_q;       // [n x k/64]
   const float *group_scale;      // [ceil(n k / 16384)]
   const uint16_t *X;             // [m x k] bf16
@@ -81,7 +83,7 @@ struct __align__(64) StreamParams {
   unsigned *err;
   int64_t n, k;
   int m, r;
-  int ntiles;                    // ceil(n / 16)
+  int ntiles;                    // ceil(n / tile rows)
   int chunks;                    // ceil((k / 64) / 4)
   int chunks_per_cta;            // chunks owned by one CTA of a cluster (<= 16)
   Nf4Tables tab;
@@ -209,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
   const uint32_t bar_w = bars + warp * kStages * 8u;                     // slot s: + 8 s
   const uint32_t ring_w = ring + warp * kStages * kCodeSlot;              // slot s: + s kCodeSlot
   const uint32_t qring_w = qring + warp * kStages * kQSlot;               // slot s: + s kQSlot
-  const int y_step = 16 * phases;
+  const int y_step = kTileRows * phases;
   // Each warp's ring starts filling before the tables are built.
   if (lane == 0) {
     for (int s = 0; s < kStages; ++s)
@@ -219,19 +221,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
   __syncwarp();
   for (int s = 0; s < kStages && s < nunits; ++s)
     issue_unit(lane == 0, bar_w + s * 8u, tx_bytes, ring_w + s * kCodeSlot, map_codes, kb0 * 32,
-               qring_w + s * kQSlot, map_q, kb0 & ~15, (t_lo + phase) * 16 + s * y_step);
+               qring_w + s * kQSlot, map_q, kb0 & ~15, (t_lo + phase) * kTileRows + s * y_step);
 
   // fp32(S / 255) of every group the CTA's rows touch.  Rows of the last
   // tile past n (codes and absmax codes read as zero) index the table too;
   // their entries repeat the last group.  Row * k/64 fits in 32 bits
   // (checked on the host).
-  const int gbase = (t_lo * 16 * kblocks) >> 8;
-  const int ngroups = ((t_hi * 16 * kblocks - 1) >> 8) - gbase + 1;
+  const int gbase = (t_lo * kTileRows * kblocks) >> 8;
+  const int ngroups = ((t_hi * kTileRows * kblocks - 1) >> 8) - gbase + 1;
   const int glast = static_cast<int>((p.n * kblocks - 1) >> 8);
   for (int i = threadIdx.x; i < ngroups; i += kThreads)
     ttab[i] = div255_rn(__ldg(p.group_scale + min(gbase + i, glast)));
   build_pair_lut(dsmem, p.tab, threadIdx.x, kThreads);
-  for (int i = threadIdx.x; i < nt * 16 * kMaxM; i += kThreads) red[i] = 0.f;
+  for (int i = threadIdx.x; i < nt * kTileRows * kMaxM; i += kThreads) red[i] = 0.f;
 
   // B operand (X): column g = 2 * token + block parity; lanes whose piece is
   // in the other block of the pair, and tokens >= m, hold zeros.
@@ -260,47 +262,46 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
     const uint32_t off_r1_p1 = off_r0_p1 + 8u * 128u;
 
     const uint32_t tab_w = smem_u32(ttab) - 4u * static_cast<uint32_t>(gbase);
-    const uint32_t qoff0 = static_cast<uint32_t>(pr) * 16u + (kb0 & 15), qoff1 = qoff0 + 8u * 16u;
+    const uint32_t qoff = static_cast<uint32_t>(pr) * 16u + (kb0 & 15);
     const uint32_t red_pred = q < p.m ? 1u : 0u;
-    // Loop state: rk = row * k/64 + kb0 for the rows pr and pr + 8 of the
-    // current tile; y_refill is the first row of the unit kStages ahead.
-    int rk0 = ((t_lo + phase) * 16 + pr) * kblocks + kb0;
-    const int rk_step = 16 * phases * kblocks, rk_8 = 8 * kblocks;
-    int y_refill = (t_lo + phase) * 16 + kStages * y_step;
-    const int y_end = t_hi * 16;
-    uint32_t red_addr = smem_u32(red) + 4u * static_cast<uint32_t>((phase * kMaxM + q) * 16 + pr);
-    const uint32_t red_step = 4u * static_cast<uint32_t>(phases * kMaxM * 16);
+    // Loop state: rk = row * k/64 + kb0 for row pr of the current tile;
+    // y_refill is the first row of the unit kStages ahead.
+    int rk0 = ((t_lo + phase) * kTileRows + pr) * kblocks + kb0;
+    const int rk_step = kTileRows * phases * kblocks, rk_8 = 8 * kblocks;
+    int y_refill = (t_lo + phase) * kTileRows + kStages * y_step;
+    const int y_end = t_hi * kTileRows;
+    uint32_t red_addr = smem_u32(red) + 4u * static_cast<uint32_t>((phase * kMaxM + q) * kTileRows + pr);
+    const uint32_t red_step = 4u * static_cast<uint32_t>(phases * kMaxM * kTileRows);
     const int nm1 = static_cast<int>(p.n) - 1;
     int u = phase;
 
     // One unit (this warp's chunk of one tile) from ring slot S; false when
-    // the warp is done or a wait gave up.
+    // the warp is done or a wait gave up.  Row pair j of the lane is rows
+    // pr + 8j of the tile (j = 0 .. 2 kSub - 1); sub-tile st holds pairs
+    // 2st and 2st + 1 and is one m16n8k16 row tile.
     const auto unit = [&](auto s_const, uint32_t ph) -> bool {
       constexpr int S = decltype(s_const)::value;
       if (u >= nt) return false;
-      const int rk1 = rk0 + rk_8;
-      uint32_t qw0 = 0, qw1 = 0;
-      float tlo0 = __uint_as_float(lds32(tab_w + 4u * static_cast<uint32_t>(rk0 >> 8)));
-      float tlo1 = __uint_as_float(lds32(tab_w + 4u * static_cast<uint32_t>(rk1 >> 8)));
-      float thi0 = tlo0, thi1 = tlo1;
-      int split0 = 4, split1 = 4;   // blocks of the chunk before each row's next group
-      if (MODE != 2) {
-        // Absmax codes by plain loads, from rows clamped to the matrix.
-        const int tile_row = (t_lo + u) * 16;
-        const int64_t bq0 = static_cast<int64_t>(min(tile_row + pr, nm1)) * kblocks + kb0;
-        const int64_t bq1 = static_cast<int64_t>(min(tile_row + pr + 8, nm1)) * kblocks + kb0;
-        if (MODE == 1) {
-          qw0 = __ldg(reinterpret_cast<const uint32_t *>(p.absmax_q + bq0));
-          qw1 = __ldg(reinterpret_cast<const uint32_t *>(p.absmax_q + bq1));
-        } else {
-          for (int b = 0; b < nvalid; ++b) {
-            qw0 |= static_cast<uint32_t>(__ldg(p.absmax_q + bq0 + b)) << (8 * b);
-            qw1 |= static_cast<uint32_t>(__ldg(p.absmax_q + bq1 + b)) << (8 * b);
+      uint32_t qw[2 * kSub];
+      float tlo[2 * kSub], thi[2 * kSub];
+      int split[2 * kSub];
+#pragma unroll
+      for (int j = 0; j < 2 * kSub; ++j) {
+        const int rk = rk0 + j * rk_8;
+        tlo[j] = __uint_as_float(lds32(tab_w + 4u * static_cast<uint32_t>(rk >> 8)));
+        thi[j] = tlo[j];
+        split[j] = 4;   // blocks of the chunk before the row's next group
+        qw[j] = 0;
+        if (MODE != 2) {
+          // Absmax codes by plain loads, from rows clamped to the matrix.
+          const int64_t bq = static_cast<int64_t>(min((t_lo + u) * kTileRows + pr + 8 * j, nm1)) * kblocks + kb0;
+          if (MODE == 1) {
+            qw[j] = __ldg(reinterpret_cast<const uint32_t *>(p.absmax_q + bq));
+          } else {
+            for (int b = 0; b < nvalid; ++b) qw[j] |= static_cast<uint32_t>(__ldg(p.absmax_q + bq + b)) << (8 * b);
+            thi[j] = __uint_as_float(lds32(tab_w + 4u * static_cast<uint32_t>((rk + nvalid - 1) >> 8)));
+            split[j] = 256 - (rk & 255);
           }
-          thi0 = __uint_as_float(lds32(tab_w + 4u * static_cast<uint32_t>((rk0 + nvalid - 1) >> 8)));
-          thi1 = __uint_as_float(lds32(tab_w + 4u * static_cast<uint32_t>((rk1 + nvalid - 1) >> 8)));
-          split0 = 256 - (rk0 & 255);
-          split1 = 256 - (rk1 & 255);
         }
       }
       // A wait that gives up (it never should) ends the warp's loop on every
@@ -311,51 +312,59 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(barp, ph, p.err, kErrTimeoutFullA))) return false;
       }
       const uint32_t slot = ring_w + S * kCodeSlot;
-      const uint4 c00 = lds128(slot + off_r0_p0), c01 = lds128(slot + off_r0_p1);
-      const uint4 c10 = lds128(slot + off_r1_p0), c11 = lds128(slot + off_r1_p1);
-      if (MODE == 2) {
-        qw0 = lds32(qring_w + S * kQSlot + qoff0);
-        qw1 = lds32(qring_w + S * kQSlot + qoff1);
+      uint4 c[kSub][4];   // [sub-tile][row g piece 0, row g piece 1, row g+8 piece 0, row g+8 piece 1]
+#pragma unroll
+      for (int st = 0; st < kSub; ++st) {
+        c[st][0] = lds128(slot + st * 2048u + off_r0_p0);
+        c[st][1] = lds128(slot + st * 2048u + off_r0_p1);
+        c[st][2] = lds128(slot + st * 2048u + off_r1_p0);
+        c[st][3] = lds128(slot + st * 2048u + off_r1_p1);
       }
-      float acc0, acc1;
+      if (MODE == 2) {
+#pragma unroll
+        for (int j = 0; j < 2 * kSub; ++j) qw[j] = lds32(qring_w + S * kQSlot + qoff + 128u * j);
+      }
+      float acc[2 * kSub];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        float d[4];
-        const uint4 cg = i == 0 ? c00 : c01, cg8 = i == 0 ? c10 : c11;
-        word_mma<true>(d, cg.x, cg8.x, lut, lane4, xf[i][0]);
-        word_mma<false>(d, cg.y, cg8.y, lut, lane4, xf[i][1]);
-        word_mma<false>(d, cg.z, cg8.z, lut, lane4, xf[i][2]);
-        word_mma<false>(d, cg.w, cg8.w, lut, lane4, xf[i][3]);
-        // d[0], d[1]: row pr, token q, blocks 2i and 2i+1; d[2], d[3]: row pr + 8.
-        const float qa0 = i == 0 ? byte_to_f32<0>(qw0) : byte_to_f32<2>(qw0);
-        const float qb0 = i == 0 ? byte_to_f32<1>(qw0) : byte_to_f32<3>(qw0);
-        const float qa1 = i == 0 ? byte_to_f32<0>(qw1) : byte_to_f32<2>(qw1);
-        const float qb1 = i == 0 ? byte_to_f32<1>(qw1) : byte_to_f32<3>(qw1);
-        if (MODE != 0) {
-          // One group per chunk: fp32(S/255) is common to the four blocks
-          // and is applied once per row below.
-          acc0 = i == 0 ? qa0 * d[0] : fmaf(qa0, d[0], acc0);
-          acc1 = i == 0 ? qa1 * d[2] : fmaf(qa1, d[2], acc1);
-          acc0 = fmaf(qb0, d[1], acc0);
-          acc1 = fmaf(qb1, d[3], acc1);
-        } else {
-          const float ta0 = 2 * i < split0 ? tlo0 : thi0, tb0 = 2 * i + 1 < split0 ? tlo0 : thi0;
-          const float ta1 = 2 * i < split1 ? tlo1 : thi1, tb1 = 2 * i + 1 < split1 ? tlo1 : thi1;
-          acc0 = i == 0 ? __fmul_rn(qa0, ta0) * d[0] : fmaf(__fmul_rn(qa0, ta0), d[0], acc0);
-          acc1 = i == 0 ? __fmul_rn(qa1, ta1) * d[2] : fmaf(__fmul_rn(qa1, ta1), d[2], acc1);
-          acc0 = fmaf(__fmul_rn(qb0, tb0), d[1], acc0);
-          acc1 = fmaf(__fmul_rn(qb1, tb1), d[3], acc1);
+        float d[kSub][4];
+#pragma unroll
+        for (int st = 0; st < kSub; ++st) {
+          const uint4 cg = c[st][i], cg8 = c[st][2 + i];
+          word_mma<true>(d[st], cg.x, cg8.x, lut, lane4, xf[i][0]);
+          word_mma<false>(d[st], cg.y, cg8.y, lut, lane4, xf[i][1]);
+          word_mma<false>(d[st], cg.z, cg8.z, lut, lane4, xf[i][2]);
+          word_mma<false>(d[st], cg.w, cg8.w, lut, lane4, xf[i][3]);
+        }
+        // d[st][0], d[st][1]: row pair 2st (row pr + 16 st), token q, blocks
+        // 2i and 2i+1; d[st][2], d[st][3]: row pair 2st + 1 (8 rows below).
+#pragma unroll
+        for (int j = 0; j < 2 * kSub; ++j) {
+          const float da = d[j >> 1][2 * (j & 1)], db = d[j >> 1][2 * (j & 1) + 1];
+          const float qa = i == 0 ? byte_to_f32<0>(qw[j]) : byte_to_f32<2>(qw[j]);
+          const float qb = i == 0 ? byte_to_f32<1>(qw[j]) : byte_to_f32<3>(qw[j]);
+          if (MODE != 0) {
+            // One group per chunk: fp32(S/255) is common to the four blocks
+            // and is applied once per row below.
+            acc[j] = i == 0 ? qa * da : fmaf(qa, da, acc[j]);
+            acc[j] = fmaf(qb, db, acc[j]);
+          } else {
+            const float ta = 2 * i < split[j] ? tlo[j] : thi[j], tb = 2 * i + 1 < split[j] ? tlo[j] : thi[j];
+            acc[j] = i == 0 ? __fmul_rn(qa, ta) * da : fmaf(__fmul_rn(qa, ta), da, acc[j]);
+            acc[j] = fmaf(__fmul_rn(qb, tb), db, acc[j]);
+          }
         }
       }
       if (MODE != 0) {
-        acc0 *= tlo0;
-        acc1 *= tlo1;
+#pragma unroll
+        for (int j = 0; j < 2 * kSub; ++j) acc[j] *= tlo[j];
       }
       // The slot's bytes are consumed: refill it with the unit kStages ahead.
       __syncwarp();
       issue_unit(lane == 0 && y_refill < y_end, bar, tx_bytes, slot, map_codes, kb0 * 32, qring_w + S * kQSlot,
                  map_q, kb0 & ~15, y_refill);
-      red_pair(red_pred, red_addr, acc0, acc1);
+#pragma unroll
+      for (int st = 0; st < kSub; ++st) red_pair(red_pred, red_addr + 64u * st, acc[2 * st], acc[2 * st + 1]);
       y_refill += y_step;
       red_addr += red_step;
       rk0 += rk_step;
@@ -386,17 +395,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
   // when this grid was not launched as its programmatic dependent).
   if (p.r > 0) asm volatile("griddepcontrol.wait;" ::: "memory");
   // CTA `crank` finishes its share of the cluster's (tile, token, row) sums.
-  const int total = nt * p.m * 16;
+  const int total = nt * p.m * kTileRows;
   const int o_lo = static_cast<int>((static_cast<int64_t>(total) * crank) / csize);
   const int o_hi = static_cast<int>((static_cast<int64_t>(total) * (crank + 1)) / csize);
   const uint32_t red_addr = smem_u32(red);
   for (int o = o_lo + static_cast<int>(threadIdx.x); o < o_hi; o += kThreads) {
-    const int ut = o / (p.m * 16);
-    const int rem = o - ut * p.m * 16;
-    const int mi = rem >> 4, rl = rem & 15;
-    const int64_t n = static_cast<int64_t>(t_lo + ut) * 16 + rl;
+    const int ut = o / (p.m * kTileRows);
+    const int rem = o - ut * p.m * kTileRows;
+    const int mi = rem / kTileRows, rl = rem % kTileRows;
+    const int64_t n = static_cast<int64_t>(t_lo + ut) * kTileRows + rl;
     if (n >= p.n) continue;
-    const uint32_t off = red_addr + static_cast<uint32_t>((ut * kMaxM + mi) * 16 + rl) * 4u;
+    const uint32_t off = red_addr + static_cast<uint32_t>((ut * kMaxM + mi) * kTileRows + rl) * 4u;
     float sum = 0.f;
     for (uint32_t peer = 0; peer < csize; ++peer) sum += ld_dsmem_f32(off, peer);
     if (p.r > 0) {
@@ -471,7 +480,7 @@ cudaError_t launch_mode(const StreamParams &p, int dev, int sms, int cs, cudaStr
 
 bool gemv_stream_supported(int64_t m, int64_t n, int64_t k) {
   // Row * k/64 indices (rows padded to whole tiles) are kept in 32 bits.
-  return m >= 1 && m <= kMaxM && k / 64 <= kMaxKBlocks && (n + 16) * (k / 64) < (int64_t(1) << 31);
+  return m >= 1 && m <= kMaxM && k / 64 <= kMaxKBlocks && (n + kTileRows) * (k / 64) < (int64_t(1) << 31);
 }
 
 cudaError_t launch_gemv_stream(const uint16_t *X, int64_t m, const uint8_t *codes, const uint8_t *absmax_q,
@@ -482,8 +491,8 @@ cudaError_t launch_gemv_stream(const uint16_t *X, int64_t m, const uint8_t *code
   const int64_t kblocks = k / 64;
   const int mode = kblocks % 16 == 0 ? 2 : (kblocks % 4 == 0 ? 1 : 0);
   StreamParams p{};
-  if (!encode_codes_map(&p.tmCodes, codes, n, k / 2, 128, 16, true)) return cudaErrorInvalidValue;
-  if (mode == 2 && !encode_codes_map(&p.tmQ, absmax_q, n, kblocks, 16, 16, false)) return cudaErrorInvalidValue;
+  if (!encode_codes_map(&p.tmCodes, codes, n, k / 2, 128, kTileRows, true)) return cudaErrorInvalidValue;
+  if (mode == 2 && !encode_codes_map(&p.tmQ, absmax_q, n, kblocks, 16, kTileRows, false)) return cudaErrorInvalidValue;
   p.absmax_q = absmax_q;
   p.group_scale = group_scale;
   p.X = X;
@@ -495,7 +504,7 @@ cudaError_t launch_gemv_stream(const uint16_t *X, int64_t m, const uint8_t *code
   p.k = k;
   p.m = static_cast<int>(m);
   p.r = (T != nullptr && B != nullptr) ? r : 0;
-  p.ntiles = static_cast<int>((n + 15) / 16);
+  p.ntiles = static_cast<int>((n + kTileRows - 1) / kTileRows);
   p.chunks = static_cast<int>((kblocks + 3) / 4);
   const int cs = (p.chunks + kWarps - 1) / kWarps;
   p.chunks_per_cta = (p.chunks + cs - 1) / cs;
