@@ -316,12 +316,15 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
   cluster_sync_all();
 }
 
-// T[m x r] = bf16(scale * X . A^T): one CTA per adapter row j.
-__global__ void __launch_bounds__(256) lora_proj_small_kernel(const uint16_t *__restrict__ X, int m,
+// T[m x r] = bf16(scale * X . A^T): one CTA per adapter row j, 1024 threads
+// so that K up to 8192 is one pass (the kernel sits on the critical path of a
+// decode call: the main kernel's CTAs cannot share an SM with it).
+constexpr int kProjThreads = 1024;
+__global__ void __launch_bounds__(kProjThreads) lora_proj_small_kernel(const uint16_t *__restrict__ X, int m,
                                                               int64_t k, const uint16_t *__restrict__ A,
                                                               int r, float scale,
                                                               uint16_t *__restrict__ T) {
-  __shared__ float red[8][kMaxM];
+  __shared__ float red[kProjThreads / 32][kMaxM];
   // The weight-streaming kernel that consumes T may start now; it waits for
   // this grid's completion before its epilogue reads T.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(256) lora_proj_small_kernel(const uint16_t *__
   float acc[kMaxM];
 #pragma unroll
   for (int i = 0; i < kMaxM; ++i) acc[i] = 0.f;
-  for (int64_t kk = static_cast<int64_t>(threadIdx.x) * 8; kk < k; kk += 256 * 8) {
+  for (int64_t kk = static_cast<int64_t>(threadIdx.x) * 8; kk < k; kk += kProjThreads * 8) {
     const uint4 av = __ldg(reinterpret_cast<const uint4 *>(arow + kk));
     const uint32_t aa[4] = {av.x, av.y, av.z, av.w};
 #pragma unroll
@@ -360,7 +363,7 @@ __global__ void __launch_bounds__(256) lora_proj_small_kernel(const uint16_t *__
   if (threadIdx.x < m) {
     float s = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) s += red[w][threadIdx.x];
+    for (int w = 0; w < kProjThreads / 32; ++w) s += red[w][threadIdx.x];
     T[static_cast<int64_t>(threadIdx.x) * r + j] = static_cast<uint16_t>(pack_bf16x2(s * scale, 0.f) & 0xFFFFu);
   }
 }
@@ -370,7 +373,7 @@ __global__ void __launch_bounds__(256) lora_proj_small_kernel(const uint16_t *__
 cudaError_t launch_lora_proj_small(const uint16_t *X, int64_t m, int64_t k, const uint16_t *A,
                                    int32_t r, float scale, uint16_t *T, cudaStream_t stream) {
   if (m <= 0 || r <= 0) return cudaSuccess;
-  lora_proj_small_kernel<<<r, 256, 0, stream>>>(X, static_cast<int>(m), k, A, r, scale, T);
+  lora_proj_small_kernel<<<r, kProjThreads, 0, stream>>>(X, static_cast<int>(m), k, A, r, scale, T);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -73,6 +73,11 @@ struct WeightView {
 cudaError_t tc_fwd(const uint16_t *X, int64_t m, const WeightView &w, const uint16_t *T,
                    const uint16_t *B, int32_t r, uint16_t *Y, cudaStream_t stream, bool pdl);
 
+// The same for m > 128: 256 x 256 tiles, separate rings for the X tile, the
+// packed codes and the dequantized weight tile (fused_fwd.cu).
+cudaError_t fused_fwd_large(const uint16_t *X, int64_t m, const WeightView &w, const uint16_t *T,
+                            const uint16_t *B, int32_t r, uint16_t *Y, cudaStream_t stream, bool pdl);
+
 // dX = bf16(dY . W^ + U . A); U may be null.
 cudaError_t tc_bwd_dx(const uint16_t *dY, int64_t m, const WeightView &w, const uint16_t *U,
                       const uint16_t *A, int32_t r, uint16_t *dX, cudaStream_t stream, bool pdl);

@@ -39,6 +39,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tcgen05.cuh"
 
 namespace qlora {
 namespace {
@@ -64,72 +65,6 @@ struct __align__(64) TcParams {
   float alpha;
   Nf4Tables tab;
 };
-
-// ---- PTX wrappers --------------------------------------------------------
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint64_t *bar, int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return static_cast<uint64_t>((addr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(lbo >> 4) << 16) |
-         (static_cast<uint64_t>(sbo >> 4) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// kind::f16 instruction descriptor: bf16 x bf16 -> fp32, M = 128.
-__host__ __device__ constexpr uint32_t make_idesc(int n, bool a_mn, bool b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
-         (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t *bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
-        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
-        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-
-__device__ __forceinline__ void sts128(uint32_t addr, const uint32_t (&v)[4]) {
-  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
-               : "memory");
-}
 
 // ---- compile-time configuration -------------------------------------------
 
@@ -347,6 +282,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
       int64_t g_cur = -1;
       float t_cur = 0.f;
       constexpr int kStride = C::DQ_GROUPS > 0 ? C::DQ_GROUPS : 1;
+      // Each stage must be taken by one group only (STAGES a multiple of the
+      // group count), so that a group waits on every phase of its stages'
+      // barriers and a parity wait cannot be satisfied by an older phase.
+      static_assert(C::DQ_GROUPS <= 1 || C::STAGES % C::DQ_GROUPS == 0, "stages per dequant group");
       for (int it = grp; it < total; it += kStride) {
         const int s = it % C::STAGES;
         const uint32_t ph = static_cast<uint32_t>(it / C::STAGES) & 1u;
@@ -559,7 +498,6 @@ int choose_split(int64_t tiles, int ksteps) {
 
 int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
-using CfgFwd2 = Cfg<256, 2, false, true, false, false>;
 using CfgFwd1 = Cfg<256, 1, false, true, false, false>;
 using CfgBwd2 = Cfg<256, 2, false, true, true, false>;
 using CfgBwd1 = Cfg<256, 1, false, true, true, false>;
@@ -572,9 +510,10 @@ using CfgTNT = Cfg<64, 1, true, false, true, true, true>;
 
 cudaError_t tc_fwd(const uint16_t *X, int64_t m, const WeightView &w, const uint16_t *T, const uint16_t *B,
                    int32_t r, uint16_t *Y, cudaStream_t stream, bool pdl) {
+  // Above 128 rows: the 256 x 256 kernel with separate operand rings.
+  if (m > 128) return fused_fwd_large(X, m, w, T, B, r, Y, stream, pdl);
   TcParams p{};
-  const bool big = m > 128;
-  const uint32_t bm = big ? 256u : 128u;
+  const uint32_t bm = 128u;
   const bool lora = T != nullptr && B != nullptr && r > 0;
   if (!encode_bf16_map(&p.tmA, X, m, w.k, 64, 128)) return cudaErrorInvalidValue;
   if (!encode_codes_map(&p.tmCodes, w.codes, w.n, w.k / 2, 32, 256, false)) return cudaErrorInvalidValue;
@@ -597,8 +536,7 @@ cudaError_t tc_fwd(const uint16_t *X, int64_t m, const WeightView &w, const uint
   p.alpha = 1.0f;
   p.tab = nf4_tables();
   const int gn = cdiv(w.n, 256), gm = cdiv(m, bm);
-  return big ? launch<CfgFwd2>(p, gn, gm, stream, 1, p.pdl != 0)
-             : launch<CfgFwd1>(p, gn, gm, stream, 1, p.pdl != 0);
+  return launch<CfgFwd1>(p, gn, gm, stream, 1, p.pdl != 0);
 }
 
 cudaError_t tc_bwd_dx(const uint16_t *dY, int64_t m, const WeightView &w, const uint16_t *U, const uint16_t *A,
