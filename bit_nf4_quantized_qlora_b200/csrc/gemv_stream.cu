@@ -223,20 +223,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
     issue_unit(lane == 0, bar_w + s * 8u, tx_bytes, ring_w + s * kCodeSlot, map_codes, kb0 * 32,
                qring_w + s * kQSlot, map_q, kb0 & ~15, (t_lo + phase) * kTileRows + s * y_step);
 
-  // fp32(S / 255) of every group the CTA's rows touch.  Rows of the last
-  // tile past n (codes and absmax codes read as zero) index the table too;
-  // their entries repeat the last group.  Row * k/64 fits in 32 bits
-  // (checked on the host).
-  const int gbase = (t_lo * kTileRows * kblocks) >> 8;
-  const int ngroups = ((t_hi * kTileRows * kblocks - 1) >> 8) - gbase + 1;
-  const int glast = static_cast<int>((p.n * kblocks - 1) >> 8);
-  for (int i = threadIdx.x; i < ngroups; i += kThreads)
-    ttab[i] = div255_rn(__ldg(p.group_scale + min(gbase + i, glast)));
-  build_pair_lut(dsmem, p.tab, threadIdx.x, kThreads);
-  for (int i = threadIdx.x; i < nt * kTileRows * kMaxM; i += kThreads) red[i] = 0.f;
-
   // B operand (X): column g = 2 * token + block parity; lanes whose piece is
-  // in the other block of the pair, and tokens >= m, hold zeros.
+  // in the other block of the pair, and tokens >= m, hold zeros.  Loaded
+  // before the tables are built so that the load latency overlaps them.
   const int tok = g >> 1;
   const bool live = active && (g & 1) == (q >> 1) && tok < p.m;
   uint4 xf[2][4];
@@ -248,6 +237,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
 #pragma unroll
     for (int j = 0; j < 4; ++j) xf[i][j] = v ? __ldg(xp + j) : make_uint4(0u, 0u, 0u, 0u);
   }
+
+  // fp32(S / 255) of every group the CTA's rows touch.  Rows of the last
+  // tile past n (codes and absmax codes read as zero) index the table too;
+  // their entries repeat the last group.  Row * k/64 fits in 32 bits
+  // (checked on the host).  The first group scale of each thread is loaded
+  // before the pair table is built.
+  const int gbase = (t_lo * kTileRows * kblocks) >> 8;
+  const int ngroups = ((t_hi * kTileRows * kblocks - 1) >> 8) - gbase + 1;
+  const int glast = static_cast<int>((p.n * kblocks - 1) >> 8);
+  const float s_first = static_cast<int>(threadIdx.x) < ngroups
+                            ? __ldg(p.group_scale + min(gbase + static_cast<int>(threadIdx.x), glast))
+                            : 0.f;
+  build_pair_lut(dsmem, p.tab, threadIdx.x, kThreads);
+  for (int i = threadIdx.x; i < nt * kTileRows * kMaxM; i += kThreads) red[i] = 0.f;
+  if (static_cast<int>(threadIdx.x) < ngroups) ttab[threadIdx.x] = div255_rn(s_first);
+  for (int i = threadIdx.x + kThreads; i < ngroups; i += kThreads)
+    ttab[i] = div255_rn(__ldg(p.group_scale + min(gbase + i, glast)));
   __syncthreads();
 
   if (active) {
