@@ -32,12 +32,15 @@ Storage format (the readings are listed where the pages are silent):
       Weights are quantized against the fp32 c_b, then the constants are
       compressed (the two-stage reading of P1 and P5).
 
+The same functions take a ``codebook`` name (``oracle.codebooks``): the FP4
+and INT4 baselines change only the sixteen levels and their midpoints.
+
 Inputs must be finite; that precondition is checked here only.
 """
 
 import numpy as np
 
-from . import nf4
+from . import codebooks, nf4
 
 BLOCK = 64
 GROUP = 256
@@ -78,14 +81,16 @@ def block_absmax(w_flat: np.ndarray) -> np.ndarray:
     return np.max(np.abs(w.reshape(-1, BLOCK)), axis=1).astype(np.float32)
 
 
-def nf4_codes(w_flat: np.ndarray, absmax: np.ndarray) -> np.ndarray:
-    """a2: one NF4 code (0..15, uint8) per weight, from the fp32 block absmax."""
+def nf4_codes(w_flat: np.ndarray, absmax: np.ndarray, codebook: str = "nf4") -> np.ndarray:
+    """a2: one code (0..15, uint8) per weight, from the fp32 block absmax; the
+    decision midpoints are those of ``codebook`` (NF4 unless a baseline of
+    ``oracle.codebooks`` is named)."""
     w = np.asarray(w_flat, dtype=np.float32).reshape(-1, BLOCK)
     c = np.asarray(absmax, dtype=np.float32).reshape(-1, 1)
     safe = np.where(c > 0, c, np.float32(1.0)).astype(np.float32)
     x = (w / safe).astype(np.float32)          # IEEE fp32 division
     x = np.where(c > 0, x, np.float32(0.0)).astype(np.float32)
-    t = nf4.midpoints_f32()
+    t = codebooks.midpoints_f32(codebook)
     codes = np.zeros(x.shape, dtype=np.uint8)
     for ti in t:                                # count of midpoints below x
         codes += (x > ti).astype(np.uint8)
@@ -126,7 +131,7 @@ def double_quantize(absmax: np.ndarray):
     return q, S
 
 
-def quantize_nf4_dq(w_flat: np.ndarray):
+def quantize_nf4_dq(w_flat: np.ndarray, codebook: str = "nf4"):
     """a1-a3 for a flat row-major weight whose length is a multiple of 64.
 
     Returns (packed codes uint8 [len/2], q uint8 [nb], S fp32 [ng],
@@ -134,7 +139,7 @@ def quantize_nf4_dq(w_flat: np.ndarray):
     slice that starts on a 16384-element boundary of a larger weight gives
     exactly that weight's groups."""
     c = block_absmax(w_flat)
-    codes = nf4_codes(w_flat, c)
+    codes = nf4_codes(w_flat, c, codebook)
     q, S = double_quantize(c)
     return pack_codes(codes), q, S, c
 
@@ -152,20 +157,20 @@ def absmax_dequant(q: np.ndarray, S: np.ndarray) -> np.ndarray:
     return (q.astype(np.float32) * t[g]).astype(np.float32)
 
 
-def dequant_f32(packed: np.ndarray, q: np.ndarray, S: np.ndarray) -> np.ndarray:
+def dequant_f32(packed: np.ndarray, q: np.ndarray, S: np.ndarray, codebook: str = "nf4") -> np.ndarray:
     """fp32(L[code] * c') for every weight, before the bf16 cast."""
     codes = unpack_codes(packed)
     cprime = absmax_dequant(q, S)
-    lv = nf4.levels_f32()
+    lv = codebooks.levels_f32(codebook)
     vals = lv[codes].reshape(-1, BLOCK)
     return (vals * cprime.reshape(-1, 1)).astype(np.float32).reshape(-1)
 
 
-def dequant_bf16_bits(packed: np.ndarray, q: np.ndarray, S: np.ndarray) -> np.ndarray:
+def dequant_bf16_bits(packed: np.ndarray, q: np.ndarray, S: np.ndarray, codebook: str = "nf4") -> np.ndarray:
     """a4: W^ as bf16 bit patterns (uint16), flat row-major."""
-    return bf16_rne_bits(dequant_f32(packed, q, S))
+    return bf16_rne_bits(dequant_f32(packed, q, S, codebook))
 
 
-def dequant_bf16_values(packed: np.ndarray, q: np.ndarray, S: np.ndarray) -> np.ndarray:
+def dequant_bf16_values(packed: np.ndarray, q: np.ndarray, S: np.ndarray, codebook: str = "nf4") -> np.ndarray:
     """a4: W^ as the fp64 values of its bf16 entries (exact)."""
-    return bf16_bits_to_f32(dequant_bf16_bits(packed, q, S)).astype(np.float64)
+    return bf16_bits_to_f32(dequant_bf16_bits(packed, q, S, codebook)).astype(np.float64)
