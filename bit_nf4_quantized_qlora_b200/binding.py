@@ -23,6 +23,13 @@ QLORA_ERR_ALIGN = -3
 QLORA_ERR_WORKSPACE = -4
 QLORA_ERR_CUDA = -5
 QLORA_ERR_DEVICE = -6
+QLORA_ERR_CODEBOOK = -7
+
+# 4-bit codebooks (the weight's `codebook`): NF4 and the FP4 / INT4 baselines.
+QLORA_CODEBOOK_NF4 = 0
+QLORA_CODEBOOK_FP4 = 1
+QLORA_CODEBOOK_INT4 = 2
+CODEBOOKS = {"nf4": QLORA_CODEBOOK_NF4, "fp4": QLORA_CODEBOOK_FP4, "int4": QLORA_CODEBOOK_INT4}
 
 QLORA_OP_FWD = 0
 QLORA_OP_BWD_DX = 1
@@ -45,7 +52,7 @@ class QLoRAError(RuntimeError):
 class NF4WeightC(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("absmax_q", ctypes.c_void_p),
                 ("group_scale", ctypes.c_void_p), ("n", ctypes.c_int64), ("k", ctypes.c_int64),
-                ("block", ctypes.c_int32), ("group", ctypes.c_int32)]
+                ("block", ctypes.c_int32), ("group", ctypes.c_int32), ("codebook", ctypes.c_int32)]
 
 
 _LIB = None
@@ -53,6 +60,10 @@ _LIB = None
 _SIGNATURES = {
     "qlora_quantize_nf4_dq": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
                                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_quantize_4bit_dq": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
+                                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                              ctypes.c_void_p]),
+    "qlora_codebook_levels": (ctypes.c_int, [ctypes.c_int32, ctypes.POINTER(ctypes.c_float)]),
     "qlora_dequant": (ctypes.c_int, [ctypes.POINTER(NF4WeightC), ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_linear_fwd": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(NF4WeightC),
                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_float,
@@ -126,10 +137,11 @@ class NF4Weight:
     group_scale: torch.Tensor    # float32 [ceil(n*k/64/256)]
     n: int
     k: int
+    codebook: int = QLORA_CODEBOOK_NF4
 
     def c_struct(self) -> NF4WeightC:
         return NF4WeightC(self.codes.data_ptr(), self.absmax_q.data_ptr(), self.group_scale.data_ptr(),
-                          self.n, self.k, BLOCK, GROUP)
+                          self.n, self.k, BLOCK, GROUP, self.codebook)
 
     @property
     def nbytes(self) -> int:
@@ -147,6 +159,12 @@ def qlora_workspace_bytes(op: int, m: int, n: int, k: int, r: int) -> int:
 def qlora_nf4_levels() -> list:
     buf = (ctypes.c_float * 16)()
     lib().qlora_nf4_levels(buf)
+    return [float(v) for v in buf]
+
+
+def qlora_codebook_levels(codebook: int) -> list:
+    buf = (ctypes.c_float * 16)()
+    _check("qlora_codebook_levels", lib().qlora_codebook_levels(codebook, buf))
     return [float(v) for v in buf]
 
 
@@ -171,6 +189,12 @@ def qlora_poll_device_error(stream=None) -> int:
 def qlora_quantize_nf4_dq(W: torch.Tensor, absmax_fp32: Optional[torch.Tensor] = None,
                           out: Optional[NF4Weight] = None, stream=None) -> NF4Weight:
     """fp32 W [n x k] on the device -> NF4Weight."""
+    return qlora_quantize_4bit_dq(W, QLORA_CODEBOOK_NF4, absmax_fp32, out, stream)
+
+
+def qlora_quantize_4bit_dq(W: torch.Tensor, codebook: int, absmax_fp32: Optional[torch.Tensor] = None,
+                           out: Optional[NF4Weight] = None, stream=None) -> NF4Weight:
+    """fp32 W [n x k] on the device -> NF4Weight in `codebook` (QLORA_CODEBOOK_*)."""
     _need_cuda(W, absmax_fp32)
     if W.dtype != torch.float32 or W.dim() != 2:
         raise ValueError("W must be a 2-D float32 tensor")
@@ -180,10 +204,12 @@ def qlora_quantize_nf4_dq(W: torch.Tensor, absmax_fp32: Optional[torch.Tensor] =
         dev = W.device
         out = NF4Weight(torch.empty(numel // 2, dtype=torch.uint8, device=dev),
                         torch.empty(numel // BLOCK, dtype=torch.uint8, device=dev),
-                        torch.empty(max(n_groups(numel), 1), dtype=torch.float32, device=dev), n, k)
-    _check("qlora_quantize_nf4_dq",
-           lib().qlora_quantize_nf4_dq(W.data_ptr(), n, k, out.codes.data_ptr(), out.absmax_q.data_ptr(),
-                                       out.group_scale.data_ptr(), _ptr(absmax_fp32), _stream(stream)))
+                        torch.empty(max(n_groups(numel), 1), dtype=torch.float32, device=dev), n, k, codebook)
+    else:
+        out.codebook = codebook
+    _check("qlora_quantize_4bit_dq",
+           lib().qlora_quantize_4bit_dq(W.data_ptr(), n, k, codebook, out.codes.data_ptr(), out.absmax_q.data_ptr(),
+                                        out.group_scale.data_ptr(), _ptr(absmax_fp32), _stream(stream)))
     return out
 
 

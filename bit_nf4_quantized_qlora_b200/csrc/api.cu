@@ -64,6 +64,7 @@ int check_weight(const qlora_nf4_weight *w, bool linear = true) {
   if (w->n <= 0 || w->k <= 0 || (w->k % 64) != 0) return QLORA_ERR_SHAPE;
   if (linear && (w->n % 8) != 0) return QLORA_ERR_SHAPE;
   if (w->block != 64 || w->group != 256) return QLORA_ERR_SHAPE;
+  if (w->codebook < 0 || w->codebook >= kCodebookCount) return QLORA_ERR_CODEBOOK;
   if (w->n > (int64_t(1) << 31) || w->k > (int64_t(1) << 31)) return QLORA_ERR_SHAPE;
   if (!aligned16(w->codes) || !aligned16(w->absmax_q) || !aligned16(w->group_scale)) return QLORA_ERR_ALIGN;
   return QLORA_OK;
@@ -81,7 +82,7 @@ int check_adapter(const uint16_t *A, const uint16_t *B, int32_t r, bool *use) {
 }
 
 WeightView view(const qlora_nf4_weight *w) {
-  return WeightView{w->codes, w->absmax_q, w->group_scale, w->n, w->k};
+  return WeightView{w->codes, w->absmax_q, w->group_scale, w->n, w->k, &codebook_tables(w->codebook)};
 }
 
 }  // namespace
@@ -107,7 +108,7 @@ using namespace qlora;
 
 extern "C" {
 
-int qlora_version(void) { return (1 << 16) | 0; }
+int qlora_version(void) { return (1 << 16) | 1; }
 
 int qlora_last_cuda_error(void) { return t_last_cuda_error; }
 
@@ -129,6 +130,7 @@ const char *qlora_status_string(int status) {
     case QLORA_ERR_WORKSPACE: return "QLORA_ERR_WORKSPACE: workspace missing or too small";
     case QLORA_ERR_CUDA: return "QLORA_ERR_CUDA: a CUDA call failed";
     case QLORA_ERR_DEVICE: return "QLORA_ERR_DEVICE: the current device is not sm_100";
+    case QLORA_ERR_CODEBOOK: return "QLORA_ERR_CODEBOOK: unknown codebook";
     default: return "unknown qlora status";
   }
 }
@@ -136,6 +138,13 @@ const char *qlora_status_string(int status) {
 void qlora_nf4_levels(float *levels) {
   if (!levels) return;
   std::memcpy(levels, nf4_tables().level, sizeof(float) * 16);
+}
+
+int qlora_codebook_levels(int32_t codebook, float *levels) {
+  if (!levels) return QLORA_ERR_NULL;
+  if (codebook < 0 || codebook >= kCodebookCount) return QLORA_ERR_CODEBOOK;
+  std::memcpy(levels, codebook_tables(codebook).level, sizeof(float) * 16);
+  return QLORA_OK;
 }
 
 size_t qlora_workspace_bytes(int op, int64_t m, int64_t n, int64_t k, int32_t r) {
@@ -151,7 +160,13 @@ size_t qlora_workspace_bytes(int op, int64_t m, int64_t n, int64_t k, int32_t r)
 
 int qlora_quantize_nf4_dq(const float *W, int64_t n, int64_t k, uint8_t *codes, uint8_t *absmax_q,
                           float *group_scale, float *absmax_fp32, qlora_stream_t stream) {
+  return qlora_quantize_4bit_dq(W, n, k, QLORA_CODEBOOK_NF4, codes, absmax_q, group_scale, absmax_fp32, stream);
+}
+
+int qlora_quantize_4bit_dq(const float *W, int64_t n, int64_t k, int32_t codebook, uint8_t *codes,
+                           uint8_t *absmax_q, float *group_scale, float *absmax_fp32, qlora_stream_t stream) {
   if (!W || !codes || !absmax_q || !group_scale) return QLORA_ERR_NULL;
+  if (codebook < 0 || codebook >= kCodebookCount) return QLORA_ERR_CODEBOOK;
   if (n <= 0 || k <= 0 || (k % 64) != 0) return QLORA_ERR_SHAPE;
   if (n > (int64_t(1) << 40) / k) return QLORA_ERR_SHAPE;
   if (!aligned16(W) || !aligned16(codes) || !aligned16(absmax_q) || !aligned16(group_scale) ||
@@ -159,7 +174,7 @@ int qlora_quantize_nf4_dq(const float *W, int64_t n, int64_t k, uint8_t *codes, 
     return QLORA_ERR_ALIGN;
   int st = check_device();
   if (st != QLORA_OK) return st;
-  return cuda_status(launch_quantize(W, n * k, codes, absmax_q, group_scale, absmax_fp32,
+  return cuda_status(launch_quantize(W, n * k, codes, absmax_q, group_scale, absmax_fp32, codebook_tables(codebook),
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -171,7 +186,7 @@ int qlora_dequant(const qlora_nf4_weight *w, uint16_t *W_bf16, qlora_stream_t st
   st = check_device();
   if (st != QLORA_OK) return st;
   return cuda_status(launch_dequant(w->codes, w->absmax_q, w->group_scale, w->n * w->k, W_bf16,
-                                    reinterpret_cast<cudaStream_t>(stream)));
+                                    codebook_tables(w->codebook), reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int qlora_linear_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w, const uint16_t *A,
@@ -206,9 +221,9 @@ int qlora_linear_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w, co
       // or K beyond one cluster's warps) the CTA-ring kernel.
       e = gemv_stream_supported(m, w->n, w->k)
               ? launch_gemv_stream(X, m, w->codes, w->absmax_q, w->group_scale, w->n, w->k, T,
-                                   lora ? B : nullptr, lora ? r : 0, Y, s, pdl)
+                                   lora ? B : nullptr, lora ? r : 0, Y, codebook_tables(w->codebook), s, pdl)
               : launch_gemv_fwd(X, m, w->codes, w->absmax_q, w->group_scale, w->n, w->k, T, lora ? B : nullptr,
-                                lora ? r : 0, Y, s, pdl);
+                                lora ? r : 0, Y, codebook_tables(w->codebook), s, pdl);
     }
   } else {
     if (lora) e = tc_proj_kmajor(X, m, w->k, A, r, scale, T, s);

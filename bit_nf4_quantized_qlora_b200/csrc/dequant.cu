@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t *__rest
 }  // namespace
 
 cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *absmax_q, const float *group_scale,
-                           int64_t numel, uint16_t *out, cudaStream_t stream) {
+                           int64_t numel, uint16_t *out, const Nf4Tables &tab, cudaStream_t stream) {
   const int64_t nh = numel / 32;
   if (nh == 0) return cudaSuccess;
   int dev = 0, sms = 148;
@@ -56,7 +56,7 @@ cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *absmax_q, const 
   const int64_t want = (nh + kThreads - 1) / kThreads;
   const int64_t cap = static_cast<int64_t>(sms) * 8;
   const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
-  dequant_kernel<<<grid, kThreads, 0, stream>>>(codes, absmax_q, group_scale, nh, out, nf4_tables());
+  dequant_kernel<<<grid, kThreads, 0, stream>>>(codes, absmax_q, group_scale, nh, out, tab);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -306,7 +306,7 @@ cudaError_t fused_fwd_large(const uint16_t *X, int64_t m, const WeightView &w, c
   p.num_main = static_cast<int>(w.k / kBK);
   p.num_lora = lora ? (r + kBK - 1) / kBK : 0;
   p.pdl = (lora && pdl) ? 1 : 0;
-  p.tab = nf4_tables();
+  p.tab = *w.tab;
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

@@ -380,7 +380,8 @@ cudaError_t launch_lora_proj_small(const uint16_t *X, int64_t m, int64_t k, cons
 
 cudaError_t launch_gemv_fwd(const uint16_t *X, int64_t m, const uint8_t *codes, const uint8_t *absmax_q,
                             const float *group_scale, int64_t n, int64_t k, const uint16_t *T,
-                            const uint16_t *B, int32_t r, uint16_t *Y, cudaStream_t stream, bool pdl) {
+                            const uint16_t *B, int32_t r, uint16_t *Y, const Nf4Tables &tab,
+                            cudaStream_t stream, bool pdl) {
   if (m <= 0) return cudaSuccess;
   GemvParams p{};
   if (!encode_codes_map(&p.tmCodes, codes, n, k / 2, 128, kRows, true)) return cudaErrorInvalidValue;
@@ -395,7 +396,7 @@ cudaError_t launch_gemv_fwd(const uint16_t *X, int64_t m, const uint8_t *codes, 
   p.k = k;
   p.m = static_cast<int>(m);
   p.r = (T != nullptr && B != nullptr) ? r : 0;
-  p.tab = nf4_tables();
+  p.tab = tab;
 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);

@@ -491,7 +491,8 @@ bool gemv_stream_supported(int64_t m, int64_t n, int64_t k) {
 
 cudaError_t launch_gemv_stream(const uint16_t *X, int64_t m, const uint8_t *codes, const uint8_t *absmax_q,
                                const float *group_scale, int64_t n, int64_t k, const uint16_t *T,
-                               const uint16_t *B, int32_t r, uint16_t *Y, cudaStream_t stream, bool pdl) {
+                               const uint16_t *B, int32_t r, uint16_t *Y, const Nf4Tables &tab,
+                               cudaStream_t stream, bool pdl) {
   if (m <= 0) return cudaSuccess;
   if (!gemv_stream_supported(m, n, k)) return cudaErrorInvalidValue;
   const int64_t kblocks = k / 64;
@@ -514,7 +515,7 @@ cudaError_t launch_gemv_stream(const uint16_t *X, int64_t m, const uint8_t *code
   p.chunks = static_cast<int>((kblocks + 3) / 4);
   const int cs = (p.chunks + kWarps - 1) / kWarps;
   p.chunks_per_cta = (p.chunks + cs - 1) / cs;
-  p.tab = nf4_tables();
+  p.tab = tab;
 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);

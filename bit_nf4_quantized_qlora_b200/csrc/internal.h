@@ -10,7 +10,9 @@
 
 namespace qlora {
 
-// The library's own NF4 codebook and midpoints (derived once at load time).
+// The library's codebooks and their midpoints (derived once at load time):
+// codebook_tables(kCodebookNF4 | kCodebookFP4 | kCodebookINT4).
+const Nf4Tables &codebook_tables(int codebook);
 const Nf4Tables &nf4_tables();
 
 // Device error word (bounded waits that gave up); one per device.
@@ -33,10 +35,10 @@ bool encode_codes_map(CUtensorMap *m, const uint8_t *ptr, int64_t rows, int64_t 
 // --- launchers (all asynchronous on `stream`; return cudaError_t) --------
 
 cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q,
-                            float *group_scale, float *absmax_fp32, cudaStream_t stream);
+                            float *group_scale, float *absmax_fp32, const Nf4Tables &tab, cudaStream_t stream);
 
 cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *absmax_q, const float *group_scale,
-                           int64_t numel, uint16_t *out, cudaStream_t stream);
+                           int64_t numel, uint16_t *out, const Nf4Tables &tab, cudaStream_t stream);
 
 // T[m x r] = bf16(scale * X[m x k] . A[r x k]^T) for small m (m <= 16).
 cudaError_t launch_lora_proj_small(const uint16_t *X, int64_t m, int64_t k, const uint16_t *A,
@@ -47,7 +49,7 @@ cudaError_t launch_lora_proj_small(const uint16_t *X, int64_t m, int64_t k, cons
 cudaError_t launch_gemv_fwd(const uint16_t *X, int64_t m, const uint8_t *codes,
                             const uint8_t *absmax_q, const float *group_scale, int64_t n, int64_t k,
                             const uint16_t *T, const uint16_t *B, int32_t r, uint16_t *Y,
-                            cudaStream_t stream, bool pdl);
+                            const Nf4Tables &tab, cudaStream_t stream, bool pdl);
 
 // Decode-sized forward (m <= 4, k/64 <= 512): per-warp TMA streams of the
 // codes, K split over a cluster.  Same contract as launch_gemv_fwd.
@@ -55,7 +57,7 @@ bool gemv_stream_supported(int64_t m, int64_t n, int64_t k);
 cudaError_t launch_gemv_stream(const uint16_t *X, int64_t m, const uint8_t *codes,
                                const uint8_t *absmax_q, const float *group_scale, int64_t n, int64_t k,
                                const uint16_t *T, const uint16_t *B, int32_t r, uint16_t *Y,
-                               cudaStream_t stream, bool pdl);
+                               const Nf4Tables &tab, cudaStream_t stream, bool pdl);
 
 // tcgen05 paths -------------------------------------------------------------
 
@@ -64,6 +66,7 @@ struct WeightView {
   const uint8_t *absmax_q;
   const float *group_scale;
   int64_t n, k;
+  const Nf4Tables *tab;   // the weight's codebook
 };
 
 // Y = bf16(X . W^T + T . B^T); T may be null (no adapter).

@@ -1,4 +1,8 @@
-// NF4 codebook of the CUDA library, derived on the host at load time.
+// Codebooks of the CUDA library, derived on the host at load time: NF4 and
+// the two uniform-bin 4-bit baselines it is compared with.
+//
+// NF4 ("QLoRA and Quantized Training", The idea; "A 65B fine-tune on the GPU
+// you already have", figure 3):
 //
 // 16 levels at quantiles of a standard normal with equal probability mass per
 // bin ("QLoRA and Quantized Training", The idea; "A 65B fine-tune on the GPU
@@ -10,6 +14,16 @@
 //
 // Phi^-1 is computed here independently: bisection on the complementary error
 // function in long double, polished by Newton steps.
+//
+// Baselines ("QLoRA Explained", The three ideas behind QLoRA: NF4 beats the
+// standard 4-bit integer and float formats on normal data; "A 65B fine-tune",
+// figure 3: their bins are uniform).  The pages do not define them; taken:
+//   FP4  the e2m1 float (sign, 2 exponent bits with bias 1, 1 mantissa bit,
+//        subnormals at exponent 0), its 16 bit patterns decoded and divided by
+//        the largest magnitude, 6; ascending, so code 7 is -0 and code 8 +0.
+//   INT4 symmetric absmax integers: i/7 for i = -7..7 at codes 0..14, code 15
+//        repeating +1 (never chosen: its midpoint with code 14 is 1).
+// Midpoints as for NF4: fp32(L_i + L_i+1) halved.
 #include <algorithm>
 #include <cmath>
 #include <mutex>
@@ -47,6 +61,37 @@ Nf4Tables build_tables() {
   const long double top = normal_quantile(o);
   Nf4Tables t{};
   for (int i = 0; i < 16; ++i) t.level[i] = static_cast<float>(static_cast<double>(v[i] / top));
+  return t;
+}
+
+// Value of the e2m1 bit pattern `b` (bit 3 sign, bits 2..1 exponent, bit 0
+// mantissa).
+double e2m1_value(int b) {
+  const int e = (b >> 1) & 3, m = b & 1;
+  const double mag = e == 0 ? 0.5 * m : std::ldexp(1.0 + 0.5 * m, e - 1);
+  return (b & 8) ? -mag : mag;
+}
+
+Nf4Tables build_fp4() {
+  // Negative patterns from the largest magnitude down to -0, then +0 up.
+  int order[16];
+  for (int i = 0; i < 8; ++i) order[i] = 15 - i;   // 1111 (-6) .. 1000 (-0)
+  for (int i = 0; i < 8; ++i) order[8 + i] = i;    // 0000 (+0) .. 0111 (+6)
+  const double top = e2m1_value(7);
+  Nf4Tables t{};
+  for (int i = 0; i < 16; ++i) t.level[i] = static_cast<float>(e2m1_value(order[i]) / top);
+  t.level[7] = -0.0f;
+  return t;
+}
+
+Nf4Tables build_int4() {
+  Nf4Tables t{};
+  for (int i = 0; i < 15; ++i) t.level[i] = static_cast<float>(static_cast<double>(i - 7) / 7.0);
+  t.level[15] = 1.0f;
+  return t;
+}
+
+Nf4Tables with_midpoints(Nf4Tables t) {
   for (int i = 0; i < 15; ++i) {
     volatile float s = t.level[i] + t.level[i + 1];  // fp32 add, then exact halving
     t.mid[i] = s * 0.5f;
@@ -57,9 +102,12 @@ Nf4Tables build_tables() {
 
 }  // namespace
 
-const Nf4Tables &nf4_tables() {
-  static const Nf4Tables tables = build_tables();
-  return tables;
+const Nf4Tables &codebook_tables(int codebook) {
+  static const Nf4Tables tables[kCodebookCount] = {with_midpoints(build_tables()), with_midpoints(build_fp4()),
+                                                   with_midpoints(build_int4())};
+  return tables[(codebook >= 0 && codebook < kCodebookCount) ? codebook : kCodebookNF4];
 }
+
+const Nf4Tables &nf4_tables() { return codebook_tables(kCodebookNF4); }
 
 }  // namespace qlora

@@ -30,7 +30,13 @@ constexpr float kMinFastAbsmax = 0x1p-100f;
 __device__ __forceinline__ float div_by_absmax(float w, float m, float y) {
   const float q0 = __fmul_rn(w, y);
   const float rho = __fmaf_rn(-q0, m, w);
-  return __fmaf_rn(rho, y, q0);
+  float x = __fmaf_rn(rho, y, q0);
+  // Below the normal range the residual can underflow and the result may be
+  // off by an ulp.  Only zero against nonzero (and the sign) can decide a
+  // code there, and only in a codebook with a midpoint at 0 (FP4: -0 | +0):
+  // IEEE division settles those rare quotients.
+  if (fabsf(x) < 0x1p-125f) x = __fdiv_rn(w, m);
+  return x;
 }
 
 // #{i : x > T_i} over the 15 sorted midpoints, as a branchless binary search:
@@ -96,7 +102,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const float *__restr
         // theorem): with y = RN(1/m) and q0 = RN(w*y) within one ulp of w/m,
         // the residual w - m*q0 is exact in one FMA and RN(q0 + residual*y)
         // is RN(w/m).  |w/m| <= 1 cannot overflow; results below the normal
-        // range all give code 7, where rounding does not matter.
+        // range are redone by IEEE division (div_by_absmax).
         const float y = __frcp_rn(m);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -157,12 +163,12 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const float *__restr
 }  // namespace
 
 cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q,
-                            float *group_scale, float *absmax_fp32, cudaStream_t stream) {
+                            float *group_scale, float *absmax_fp32, const Nf4Tables &tab, cudaStream_t stream) {
   const int64_t nb = numel / 64;
   const int64_t ng = (nb + kBlocksPerGroup - 1) / kBlocksPerGroup;
   if (ng == 0) return cudaSuccess;
   quantize_kernel<<<static_cast<unsigned>(ng), kThreads, 0, stream>>>(W, nb, codes, absmax_q, group_scale,
-                                                                      absmax_fp32, nf4_tables());
+                                                                      absmax_fp32, tab);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -534,7 +534,7 @@ cudaError_t tc_fwd(const uint16_t *X, int64_t m, const WeightView &w, const uint
   p.num_lora = lora ? cdiv(r, 64) : 0;
   p.pdl = (lora && pdl) ? 1 : 0;
   p.alpha = 1.0f;
-  p.tab = nf4_tables();
+  p.tab = *w.tab;
   const int gn = cdiv(w.n, 256), gm = cdiv(m, bm);
   return launch<CfgFwd1>(p, gn, gm, stream, 1, p.pdl != 0);
 }
@@ -564,7 +564,7 @@ cudaError_t tc_bwd_dx(const uint16_t *dY, int64_t m, const WeightView &w, const 
   p.num_lora = lora ? cdiv(r, 64) : 0;
   p.pdl = (lora && pdl) ? 1 : 0;
   p.alpha = 1.0f;
-  p.tab = nf4_tables();
+  p.tab = *w.tab;
   const int gn = cdiv(w.k, 256), gm = cdiv(m, bm);
   return big ? launch<CfgBwd2>(p, gn, gm, stream, 1, p.pdl != 0)
              : launch<CfgBwd1>(p, gn, gm, stream, 1, p.pdl != 0);

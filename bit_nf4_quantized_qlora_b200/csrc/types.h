@@ -5,6 +5,10 @@
 
 namespace qlora {
 
+// The 4-bit codebooks a weight may be stored in (NF4, or one of the two
+// uniform-bin baselines it is compared with).
+enum : int { kCodebookNF4 = 0, kCodebookFP4 = 1, kCodebookINT4 = 2, kCodebookCount = 3 };
+
 // The fp32 codebook and the 15 decision midpoints, passed by value as a
 // kernel parameter (uniform across the grid).
 struct Nf4Tables {

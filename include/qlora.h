@@ -60,19 +60,37 @@ enum qlora_status {
   QLORA_ERR_ALIGN = -3,     /* a pointer is not 16-byte aligned            */
   QLORA_ERR_WORKSPACE = -4, /* workspace missing or smaller than required  */
   QLORA_ERR_CUDA = -5,      /* a CUDA call failed (see last_cuda_error)    */
-  QLORA_ERR_DEVICE = -6     /* the current device is not sm_100            */
+  QLORA_ERR_DEVICE = -6,    /* the current device is not sm_100            */
+  QLORA_ERR_CODEBOOK = -7   /* codebook id not one of qlora_codebook       */
 };
 
-/* Quantized weight: three flat buffers plus the shape.
- *   codes       uint8 [n*k/2]   NF4 codes, two per byte in row-major element
+/* The sixteen 4-bit values a weight's codes index.  NF4 is the method's own
+ * ("QLoRA and Quantized Training", The idea; "A 65B fine-tune on the GPU you
+ * already have", figure 3).  FP4 and INT4 are the uniform-bin baselines the
+ * pages say NF4 beats on normally distributed weights ("QLoRA Explained", The
+ * three ideas behind QLoRA; "A 65B fine-tune", figure 3); the pages do not
+ * define them, and these are the formats taken:
+ *   QLORA_CODEBOOK_FP4   e2m1 float (1 sign, 2 exponent bits with bias 1,
+ *                        1 mantissa bit): magnitudes 0 .. 6 divided by 6,
+ *                        ascending; code 7 is -0, code 8 is +0.
+ *   QLORA_CODEBOOK_INT4  symmetric integers i/7, i = -7..7, at codes 0..14;
+ *                        code 15 repeats +1 and is never produced.
+ * Every codebook is used with the same blocks, double quantization and
+ * decision rule; only the levels and their midpoints change.               */
+enum qlora_codebook { QLORA_CODEBOOK_NF4 = 0, QLORA_CODEBOOK_FP4 = 1, QLORA_CODEBOOK_INT4 = 2 };
+
+/* Quantized weight: three flat buffers plus the shape and the codebook.
+ *   codes       uint8 [n*k/2]   4-bit codes, two per byte in row-major element
  *                               order: byte j = (code[2j] << 4) | code[2j+1]
  *   absmax_q    uint8 [n*k/64]  8-bit code of each block's absmax
  *   group_scale fp32  [ceil(n*k/64/256)]  max absmax of each group of 256
  *   block == 64 and group == 256 are the only supported values.
+ *   codebook    qlora_codebook the codes index (0 == NF4, so a zeroed field
+ *               means NF4); any other value gives QLORA_ERR_CODEBOOK.
  * Dequantization ["A 65B fine-tune on the GPU you already have", figure 4;
  * "QLoRA", Storage precision is not calculation precision]:
  *   c'  = fp32(float(absmax_q[b]) * fp32(group_scale[b/256] / 255))
- *   W^  = bf16_rne(fp32(NF4[code] * c'))                                   */
+ *   W^  = bf16_rne(fp32(L[code] * c')), L the weight's codebook            */
 typedef struct {
   const uint8_t *codes;
   const uint8_t *absmax_q;
@@ -80,6 +98,7 @@ typedef struct {
   int64_t n, k;
   int32_t block;
   int32_t group;
+  int32_t codebook;
 } qlora_nf4_weight;
 
 /* Operation ids for qlora_workspace_bytes. */
@@ -104,6 +123,13 @@ enum qlora_op { QLORA_OP_FWD = 0, QLORA_OP_BWD_DX = 1, QLORA_OP_LORA_BWD = 2 };
 int qlora_quantize_nf4_dq(const float *W, int64_t n, int64_t k,
                           uint8_t *codes, uint8_t *absmax_q, float *group_scale,
                           float *absmax_fp32, qlora_stream_t stream);
+
+/* The same quantization with the levels and midpoints of `codebook`
+ * (qlora_codebook); qlora_quantize_nf4_dq is codebook QLORA_CODEBOOK_NF4.
+ * The weight it fills is used with that codebook in qlora_nf4_weight.     */
+int qlora_quantize_4bit_dq(const float *W, int64_t n, int64_t k, int32_t codebook,
+                           uint8_t *codes, uint8_t *absmax_q, float *group_scale,
+                           float *absmax_fp32, qlora_stream_t stream);
 
 /* Standalone dequantization to bf16 ["QLoRA", Storage precision is not
  * calculation precision; "A 65B fine-tune on the GPU you already have",
@@ -218,6 +244,10 @@ const char *qlora_status_string(int status);
  * quantile construction (16 ascending levels, index 7 == 0, 0 == -1,
  * 15 == +1).  Host function; writes 16 floats to `levels` (host memory).   */
 void qlora_nf4_levels(float *levels);
+
+/* The 16 fp32 levels of `codebook` in code order (host function, host
+ * memory); QLORA_ERR_CODEBOOK for an unknown id, QLORA_ERR_NULL for NULL. */
+int qlora_codebook_levels(int32_t codebook, float *levels);
 
 /* ABI version: (major << 16) | minor. */
 int qlora_version(void);

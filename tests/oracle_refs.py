@@ -16,9 +16,9 @@ def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").to(torch.float32).numpy().astype(np.float64)
 
 
-def quantize(W: torch.Tensor):
+def quantize(W: torch.Tensor, codebook: str = "nf4"):
     """Oracle quantization of a whole fp32 weight: (packed, q, S)."""
-    packed, q, S, _ = quant.quantize_nf4_dq(W.reshape(-1).numpy())
+    packed, q, S, _ = quant.quantize_nf4_dq(W.reshape(-1).numpy(), codebook)
     return packed, q, S
 
 
@@ -50,9 +50,9 @@ def dequant_rows(W: torch.Tensor, rows) -> np.ndarray:
     return res
 
 
-def dequant_full(W: torch.Tensor) -> np.ndarray:
-    p, q, S = quantize(W)
-    return quant.dequant_bf16_values(p, q, S).reshape(W.shape)
+def dequant_full(W: torch.Tensor, codebook: str = "nf4") -> np.ndarray:
+    p, q, S = quantize(W, codebook)
+    return quant.dequant_bf16_values(p, q, S, codebook).reshape(W.shape)
 
 
 def fwd(X, W_hat, A, B, s):

@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 
 from bit_nf4_quantized_qlora_b200 import binding as B
-from oracle import nf4
+from oracle import codebooks, nf4
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER_DIR = os.path.join(ROOT, "include")
@@ -52,6 +52,33 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, n)
 
 
+@pytest.mark.parametrize("name", ["nf4", "fp4", "int4"])
+def test_library_baseline_codebooks_equal_the_oracle(lib, name):
+    """The library builds each codebook with its own code (FP4 by decoding the
+    e2m1 bit patterns); levels equal the oracle's bit for bit, -0 included."""
+    got = np.array(B.qlora_codebook_levels(B.CODEBOOKS[name]), dtype=np.float32)
+    assert np.array_equal(got.view(np.uint32), codebooks.levels_f32(name).view(np.uint32))
+
+
+def test_unknown_codebook_is_rejected_on_the_host(lib):
+    buf = (ctypes.c_float * 16)()
+    assert lib.qlora_codebook_levels(3, buf) == B.QLORA_ERR_CODEBOOK
+    assert lib.qlora_codebook_levels(-1, buf) == B.QLORA_ERR_CODEBOOK
+    assert lib.qlora_quantize_4bit_dq(P, 64, 64, 3, P, P, P, None, None) == B.QLORA_ERR_CODEBOOK
+    w = _w()
+    w.codebook = 7
+    assert lib.qlora_dequant(ctypes.byref(w), P, None) == B.QLORA_ERR_CODEBOOK
+    assert _fwd(lib, w=w) == B.QLORA_ERR_CODEBOOK
+
+
+def test_weight_struct_layout():
+    """Three pointers and two int64 sizes (40 bytes), then block, group and
+    codebook (int32), padded to 8 bytes: a zeroed codebook field means NF4."""
+    assert ctypes.sizeof(B.NF4WeightC) == 56
+    assert B.NF4WeightC.codebook.offset == 48
+    assert B.NF4WeightC(0, 0, 0, 1, 64, 64, 256).codebook == B.QLORA_CODEBOOK_NF4
+
+
 def test_library_codebook_equals_oracle_codebook(lib):
     """The library derives its levels with its own inverse-normal routine; the
     fp32 values must equal the oracle's bit for bit."""
@@ -61,7 +88,7 @@ def test_library_codebook_equals_oracle_codebook(lib):
 
 def test_version_and_status_strings(lib):
     assert lib.qlora_version() >> 16 == 1
-    for st in (0, -1, -2, -3, -4, -5, -6):
+    for st in (0, -1, -2, -3, -4, -5, -6, -7):
         assert lib.qlora_status_string(st)
 
 
