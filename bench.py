@@ -390,6 +390,45 @@ def _unfused_comparator(p, dev, reps: int = 10):
     return out
 
 
+def _codebook_error(dev, reps: int = 5):
+    """Round-trip error of the library's quantize -> dequant for each 4-bit
+    codebook (NF4 and the FP4 / INT4 baselines) on a 4096x4096 N(0, 0.02)
+    weight, and on the same weight with 0.1 % of its entries at +-20 sigma;
+    plus the quantize kernel time per codebook (the same kernel, a different
+    table).  Error statistics are measured over the whole weight with torch
+    reductions on the device."""
+    import torch
+    from bit_nf4_quantized_qlora_b200 import binding as B
+    from bit_nf4_quantized_qlora_b200 import workloads as WL
+    out = {}
+    for label, frac in (("normal", 0.0), ("outliers_0.1pct_20sigma", 0.001)):
+        W = WL.weight(4096, 4096, 0.02, seed=4242, outlier_frac=frac, outlier_sigma=20.0).to(dev)
+        row = {}
+        for name, cb in B.CODEBOOKS.items():
+            w = B.qlora_quantize_4bit_dq(W, cb)
+            for _ in range(2):
+                B.qlora_quantize_4bit_dq(W, cb, out=w)
+            torch.cuda.synchronize()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record()
+            for _ in range(reps):
+                B.qlora_quantize_4bit_dq(W, cb, out=w)
+            t1.record()
+            torch.cuda.synchronize()
+            back = B.qlora_dequant(w).float()
+            err = back - W
+            row[name] = {"mse": float((err * err).mean()), "max_abs": float(err.abs().max()),
+                         "quantize_us": round(t0.elapsed_time(t1) * 1e3 / reps, 1)}
+            del w, back, err
+        for name in ("fp4", "int4"):
+            row[name]["mse_vs_nf4"] = round(row[name]["mse"] / row["nf4"]["mse"], 3)
+        out[label] = row
+        del W
+    out["workload"] = "W [4096 x 4096] fp32 ~ N(0, 0.02), block 64, 8-bit double quantization per 256 blocks"
+    torch.cuda.empty_cache()
+    return out
+
+
 def _cpu_baseline(rank: int, world: int):
     if rank != 0 or world != 1:
         return None
@@ -475,6 +514,7 @@ def run_ours(args):
     m1 = _m1_decode(dev, peaks, peak_kind) if rank == 0 else None
     layer = _decoder_layer(dev) if rank == 0 else None
     unfused = _unfused_comparator(projs[0], dev) if rank == 0 else None
+    codebook = _codebook_error(dev) if rank == 0 else None
     cpu = _cpu_baseline(rank, world)
 
     if rank == 0:
@@ -495,6 +535,7 @@ def run_ours(args):
             "m1_decode": m1,
             "decoder_layer_7b": layer,
             "unfused_comparator": unfused,
+            "codebook_error": codebook,
             "device_error_flags": dev_err,
         }
         print(json.dumps(line))
