@@ -23,6 +23,8 @@ Modules:
                  dequantization, bf16 rounding.
 * ``linear``  -- forward / backward of Y = X.dequant(W)^T + s.(X.A^T).B^T.
 * ``memory``  -- bytes-per-parameter arithmetic of the storage format.
+* ``codebooks`` -- the FP4 and INT4 baselines beside NF4.
+* ``merge``   -- folding the adapter into the dequantized base (export).
 
 Every function is pinned by a ``-m "not gpu"`` test in ``tests/test_oracle.py``
 against invariants, closed forms, brute force or a library routine; none is
