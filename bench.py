@@ -390,6 +390,53 @@ def _unfused_comparator(p, dev, reps: int = 10):
     return out
 
 
+def _merge_export(dev, peaks, peak_kind, reps: int = 10):
+    """Adapter merge W' = W^ + s B A of the 7B MLP gate weight [11008 x 4096],
+    LoRA r=64: device time per call for the bf16 export and the fp32 export,
+    as algorithmic GB/s (codes, absmax codes, group scales, A, B read; W'
+    written) against the measured HBM bandwidth.  Inputs and outputs exceed
+    L2 between calls (weight copies rotate)."""
+    import torch
+    from bit_nf4_quantized_qlora_b200 import binding as B
+    from bit_nf4_quantized_qlora_b200 import workloads as WL
+    c = WL.mlp_7b("gate")
+    w0 = B.qlora_quantize_nf4_dq(c.W().to(dev))
+    ws = [w0] + [B.NF4Weight(w0.codes.clone(), w0.absmax_q.clone(), w0.group_scale.clone(), c.n, c.k)
+                 for _ in range(3)]
+    A, Bm = c.A().to(dev), c.B().to(dev)
+    numel = c.n * c.k
+    read = weight_bytes(c.n, c.k) + 2 * c.r * (c.n + c.k)
+    out = {}
+    for name, esize in (("bf16", 2), ("fp32", 4)):
+        dst = [torch.empty(c.n, c.k, dtype=torch.bfloat16 if esize == 2 else torch.float32, device=dev)
+               for _ in range(2)]
+
+        def call(i):
+            o = dst[i % 2]
+            if esize == 2:
+                B.qlora_merge_adapter(ws[i % len(ws)], A, Bm, c.r, c.scale, out_bf16=o, want_bf16=False)
+            else:
+                B.qlora_merge_adapter(ws[i % len(ws)], A, Bm, c.r, c.scale, out_f32=o, want_bf16=False)
+        for i in range(3):
+            call(i)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for i in range(reps):
+            call(i)
+        t1.record()
+        torch.cuda.synchronize()
+        t = t0.elapsed_time(t1) * 1e-3 / reps
+        gbs = (read + esize * numel) / t / 1e9
+        out[name] = {"us": round(t * 1e6, 1), "gbps": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                     "peak_kind": peak_kind}
+        del dst
+    out["workload"] = f"merge W' = W^ + s B A, W [{c.n} x {c.k}] NF4, LoRA r={c.r}; export bf16 or fp32"
+    del ws, w0
+    torch.cuda.empty_cache()
+    return out
+
+
 def _codebook_error(dev, reps: int = 5):
     """Round-trip error of the library's quantize -> dequant for each 4-bit
     codebook (NF4 and the FP4 / INT4 baselines) on a 4096x4096 N(0, 0.02)
@@ -515,6 +562,7 @@ def run_ours(args):
     layer = _decoder_layer(dev) if rank == 0 else None
     unfused = _unfused_comparator(projs[0], dev) if rank == 0 else None
     codebook = _codebook_error(dev) if rank == 0 else None
+    merged = _merge_export(dev, peaks, peak_kind) if rank == 0 else None
     cpu = _cpu_baseline(rank, world)
 
     if rank == 0:
@@ -536,6 +584,7 @@ def run_ours(args):
             "decoder_layer_7b": layer,
             "unfused_comparator": unfused,
             "codebook_error": codebook,
+            "merge_export": merged,
             "device_error_flags": dev_err,
         }
         print(json.dumps(line))

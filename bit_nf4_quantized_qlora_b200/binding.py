@@ -65,6 +65,9 @@ _SIGNATURES = {
                                               ctypes.c_void_p]),
     "qlora_codebook_levels": (ctypes.c_int, [ctypes.c_int32, ctypes.POINTER(ctypes.c_float)]),
     "qlora_dequant": (ctypes.c_int, [ctypes.POINTER(NF4WeightC), ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_merge_adapter": (ctypes.c_int, [ctypes.POINTER(NF4WeightC), ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.c_void_p]),
     "qlora_linear_fwd": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(NF4WeightC),
                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_float,
                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
@@ -221,6 +224,24 @@ def qlora_dequant(w: NF4Weight, out: Optional[torch.Tensor] = None, stream=None)
     ws = w.c_struct()
     _check("qlora_dequant", lib().qlora_dequant(ctypes.byref(ws), out.data_ptr(), _stream(stream)))
     return out
+
+
+def qlora_merge_adapter(w: NF4Weight, A: Optional[torch.Tensor], B: Optional[torch.Tensor], r: int,
+                        scale: float, out_bf16: Optional[torch.Tensor] = None, out_f32: Optional[torch.Tensor] = None,
+                        want_bf16: bool = True, want_f32: bool = False, stream=None):
+    """W' = W^ + scale . B . A [n x k]; returns (bf16 or None, fp32 or None)."""
+    A, B, r = _lora_args(A, B, r)
+    dev = w.codes.device
+    if out_bf16 is None and want_bf16:
+        out_bf16 = torch.empty(w.n, w.k, dtype=torch.bfloat16, device=dev)
+    if out_f32 is None and want_f32:
+        out_f32 = torch.empty(w.n, w.k, dtype=torch.float32, device=dev)
+    _need_cuda(A, B, out_bf16, out_f32)
+    ws = w.c_struct()
+    _check("qlora_merge_adapter",
+           lib().qlora_merge_adapter(ctypes.byref(ws), _ptr(A), _ptr(B), r, float(scale), _ptr(out_bf16),
+                                     _ptr(out_f32), _stream(stream)))
+    return out_bf16, out_f32
 
 
 def _lora_args(A, B, r):

@@ -178,6 +178,21 @@ int qlora_quantize_4bit_dq(const float *W, int64_t n, int64_t k, int32_t codeboo
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int qlora_merge_adapter(const qlora_nf4_weight *w, const uint16_t *A, const uint16_t *B, int32_t r, float scale,
+                        uint16_t *W_bf16, float *W_f32, qlora_stream_t stream) {
+  int st = check_weight(w, false);
+  if (st != QLORA_OK) return st;
+  if (!W_bf16 && !W_f32) return QLORA_ERR_NULL;
+  if ((W_bf16 && !aligned16(W_bf16)) || (W_f32 && !aligned16(W_f32))) return QLORA_ERR_ALIGN;
+  bool lora = false;
+  st = check_adapter(A, B, r, &lora);
+  if (st != QLORA_OK) return st;
+  st = check_device();
+  if (st != QLORA_OK) return st;
+  return cuda_status(launch_merge(view(w), lora ? A : nullptr, lora ? B : nullptr, lora ? r : 0, scale, W_bf16,
+                                  W_f32, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int qlora_dequant(const qlora_nf4_weight *w, uint16_t *W_bf16, qlora_stream_t stream) {
   int st = check_weight(w, false);
   if (st != QLORA_OK) return st;

@@ -85,6 +85,11 @@ cudaError_t fused_fwd_large(const uint16_t *X, int64_t m, const WeightView &w, c
 cudaError_t tc_bwd_dx(const uint16_t *dY, int64_t m, const WeightView &w, const uint16_t *U,
                       const uint16_t *A, int32_t r, uint16_t *dX, cudaStream_t stream, bool pdl);
 
+// Adapter merge W' = W^ + scale * B . A (B [n x r], A [r x k], r % 16 == 0,
+// r <= 256; r == 0 gives W^), written as bf16 and/or fp32 [n x k].
+cudaError_t launch_merge(const WeightView &w, const uint16_t *A, const uint16_t *B, int32_t r, float scale,
+                         uint16_t *out_bf16, float *out_f32, cudaStream_t stream);
+
 // out[m x r] = bf16(scale * L[m x kc] . R^T) with R given as [r x kc] (k-major).
 cudaError_t tc_proj_kmajor(const uint16_t *L, int64_t m, int64_t kc, const uint16_t *R, int32_t r,
                            float scale, uint16_t *out, cudaStream_t stream);

@@ -26,7 +26,7 @@ WORKLOADS = {
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=("quantize", "dequant", "fwd", "fwd_nolora", "bwd_dx", "lora_bwd"), required=True)
+    ap.add_argument("--op", choices=("quantize", "dequant", "fwd", "fwd_nolora", "bwd_dx", "lora_bwd", "merge"), required=True)
     ap.add_argument("--workload", choices=sorted(WORKLOADS), required=True)
     ap.add_argument("--m", type=int, default=4096)
     ap.add_argument("--iters", type=int, default=3)
@@ -47,7 +47,7 @@ def main(argv=None):
     if a.op in ("bwd_dx", "lora_bwd"):
         dY = case.dY().to(dev)
     A, Bm = case.A().to(dev), case.B().to(dev)
-    out_w = torch.empty(case.n, case.k, dtype=torch.bfloat16, device=dev) if a.op == "dequant" else None
+    out_w = torch.empty(case.n, case.k, dtype=torch.bfloat16, device=dev) if a.op in ("dequant", "merge") else None
     if a.op in ("fwd", "fwd_nolora"):
         Y = torch.empty(case.m, case.n, dtype=torch.bfloat16, device=dev)
     if a.op == "bwd_dx":
@@ -58,6 +58,8 @@ def main(argv=None):
             B.qlora_quantize_nf4_dq(W, out=w)
         elif a.op == "dequant":
             B.qlora_dequant(w, out=out_w)
+        elif a.op == "merge":
+            B.qlora_merge_adapter(w, A, Bm, r, case.scale, out_bf16=out_w)
         elif a.op == "fwd":
             B.qlora_linear_fwd(X, w, A, Bm, r, case.scale, out=Y)
         elif a.op == "fwd_nolora":

@@ -138,6 +138,22 @@ int qlora_quantize_4bit_dq(const float *W, int64_t n, int64_t k, int32_t codeboo
  *   W_bf16  out  bf16 [n x k], bit-exact W^ as defined at qlora_nf4_weight. */
 int qlora_dequant(const qlora_nf4_weight *w, uint16_t *W_bf16, qlora_stream_t stream);
 
+/* Adapter merge (export): W' = W^ + s . B . A
+ * ["QLoRA", Training setup versus deployment setup (serve the quantized base
+ *  with the adapter, or merge into another checkpoint); Common misconception
+ *  (LoRA's matrices merge back into the frozen weight)]
+ *   w       in   quantized weight [n x k] (any codebook)
+ *   A, B    in   bf16 [r x k], [n x r]; NULL/NULL or r == 0: W' = W^ bit for
+ *                bit (FP4's -0 level included)
+ *   scale   in   s = alpha / r
+ *   W_bf16  out  bf16 [n x k] = bf16_rne(W'), or NULL
+ *   W_f32   out  fp32 [n x k] = W', or NULL (e.g. to re-quantize it with
+ *                qlora_quantize_4bit_dq into a new 4-bit checkpoint)
+ * At least one output.  W' = fma(s, acc, W^) in fp32, acc the fp32 sum of the
+ * rank-r product; W^ exactly as qlora_dequant returns it.                   */
+int qlora_merge_adapter(const qlora_nf4_weight *w, const uint16_t *A, const uint16_t *B, int32_t r,
+                        float scale, uint16_t *W_bf16, float *W_f32, qlora_stream_t stream);
+
 /* Forward: Y = bf16( X . W^T + T . B^T ),  T = bf16(s . X . A^T)
  * ["QLoRA and Quantized Training", The idea (compute in bf16, each block
  *  dequantized, used, discarded); "A 65B fine-tune on the GPU you already

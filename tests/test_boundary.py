@@ -71,6 +71,21 @@ def test_unknown_codebook_is_rejected_on_the_host(lib):
     assert _fwd(lib, w=w) == B.QLORA_ERR_CODEBOOK
 
 
+def test_merge_rejects_bad_arguments(lib):
+    w = _w()
+    f = lib.qlora_merge_adapter
+    assert f(ctypes.byref(w), P, P, 16, 2.0, None, None, None) == B.QLORA_ERR_NULL       # no output
+    assert f(ctypes.byref(w), P, P, 16, 2.0, MIS, None, None) == B.QLORA_ERR_ALIGN
+    assert f(ctypes.byref(w), P, P, 16, 2.0, None, MIS, None) == B.QLORA_ERR_ALIGN
+    assert f(ctypes.byref(w), P, P, 24, 2.0, P, None, None) == B.QLORA_ERR_SHAPE         # r % 16
+    assert f(ctypes.byref(w), P, P, 272, 2.0, P, None, None) == B.QLORA_ERR_SHAPE        # r > 256
+    assert f(ctypes.byref(w), P, None, 16, 2.0, P, None, None) == B.QLORA_ERR_NULL       # half an adapter
+    assert f(ctypes.byref(w), MIS, P, 16, 2.0, P, None, None) == B.QLORA_ERR_ALIGN
+    assert f(ctypes.byref(_w(k=1000)), P, P, 16, 2.0, P, None, None) == B.QLORA_ERR_SHAPE
+    w.codebook = 5
+    assert f(ctypes.byref(w), P, P, 16, 2.0, P, None, None) == B.QLORA_ERR_CODEBOOK
+
+
 def test_weight_struct_layout():
     """Three pointers and two int64 sizes (40 bytes), then block, group and
     codebook (int32), padded to 8 bytes: a zeroed codebook field means NF4."""
