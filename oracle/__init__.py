@@ -25,6 +25,7 @@ Modules:
 * ``memory``  -- bytes-per-parameter arithmetic of the storage format.
 * ``codebooks`` -- the FP4 and INT4 baselines beside NF4.
 * ``merge``   -- folding the adapter into the dequantized base (export).
+* ``dropout`` -- LoRA dropout on the adapter input (Philox4x64-10 mask).
 
 Every function is pinned by a ``-m "not gpu"`` test in ``tests/test_oracle.py``
 against invariants, closed forms, brute force or a library routine; none is
