@@ -225,8 +225,6 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(const __grid_constant__
 
 }  // namespace
 
-size_t merge_smem_bytes(int r) { return Layout(r).total; }
-
 cudaError_t launch_merge(const WeightView &w, const uint16_t *A, const uint16_t *B, int32_t r, float scale,
                          uint16_t *out_bf16, float *out_f32, cudaStream_t stream) {
   if (r < 0 || r > kMaxR || r % 16 != 0) return cudaErrorInvalidValue;

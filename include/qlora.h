@@ -19,6 +19,12 @@
  *     gradient flows through the frozen dequantized weight ["QLoRA", Follow
  *     one QLoRA training step; "QLoRA Explained", What is QLoRA?].
  *
+ * Entry points: qlora_quantize_nf4_dq / qlora_quantize_4bit_dq (fp32 W ->
+ * codes), qlora_dequant (codes -> bf16 W^), qlora_linear_fwd (and its
+ * _noalloc form), qlora_linear_bwd_dx, qlora_lora_bwd (adapter gradients),
+ * qlora_merge_adapter (W^ + s B A for export); helpers for workspace sizes,
+ * codebook levels, errors, versions and launch counts.
+ *
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE pointers, allocated and owned by the
  *     caller.  The library never allocates, frees or retains memory; scratch
