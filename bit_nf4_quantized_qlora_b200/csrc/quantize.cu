@@ -21,11 +21,15 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kBlocksPerGroup = 256;
-constexpr int kUnroll = 4;
-
-// Absmax values below this take the IEEE division path (1/m stays finite and
-// normal far above it).
-constexpr float kMinFastAbsmax = 0x1p-100f;
+// Absmax values below this take the IEEE division path.  The reciprocal
+// step below needs the residual w - m * q0 to be exact: its lowest bit,
+// 2^(e_m + e_q0 - 46), must not fall under the smallest subnormal 2^-149.
+// A code can only change where x = w / m is near a midpoint, |x| >= 1/24
+// (FP4's smallest nonzero one; NF4's and INT4's are larger), so e_q0 >= -5
+// there and m >= 2^-98 suffices; the guard keeps a margin.  (Quotients under
+// the normal range, where only x = 0 against x > 0 matters, are redone
+// separately in div_by_absmax.)
+constexpr float kMinFastAbsmax = 0x1p-90f;
 
 __device__ __forceinline__ float div_by_absmax(float w, float m, float y) {
   const float q0 = __fmul_rn(w, y);
