@@ -49,9 +49,20 @@ class QLoRALinear(torch.nn.Module):
         self.B = torch.nn.Parameter(Bm.to(torch.bfloat16).contiguous())
 
     @classmethod
-    def from_float(cls, W: torch.Tensor, A: torch.Tensor, Bm: torch.Tensor, alpha: float) -> "QLoRALinear":
-        """Quantize an fp32 weight [n x k] on its device (libqlora's quantize kernel)."""
-        return cls(B.qlora_quantize_nf4_dq(W.float().contiguous()), A, Bm, alpha)
+    def from_float(cls, W: torch.Tensor, A: torch.Tensor, Bm: torch.Tensor, alpha: float,
+                   codebook: int = B.QLORA_CODEBOOK_NF4) -> "QLoRALinear":
+        """Quantize an fp32 weight [n x k] on its device (libqlora's quantize
+        kernel), NF4 unless another codebook (B.QLORA_CODEBOOK_*) is named."""
+        return cls(B.qlora_quantize_4bit_dq(W.float().contiguous(), codebook), A, Bm, alpha)
+
+    @torch.no_grad()
+    def merged_weight(self, dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+        """W' = W^ + s . B . A [n x k] (bf16 or fp32) for export or serving
+        without the adapter (libqlora's merge kernel)."""
+        want_f32 = dtype == torch.float32
+        h, f = B.qlora_merge_adapter(self.w, self.A.detach(), self.B.detach(), self.r, self.scale,
+                                     want_bf16=not want_f32, want_f32=want_f32)
+        return f if want_f32 else h
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:
         lead = x.shape[:-1]

@@ -16,6 +16,7 @@ import torch
 
 import oracle_refs as R
 from bit_nf4_quantized_qlora_b200 import layer as L
+from bit_nf4_quantized_qlora_b200 import binding as B
 from bit_nf4_quantized_qlora_b200 import workloads as WL
 
 pytestmark = pytest.mark.gpu
@@ -103,3 +104,24 @@ def test_decoder_block_forward_and_adapter_gradients():
         errs["dB_" + name] = _err(block.lin[name].B.grad, ref_lins[name].B.grad)
     assert errs["out"] <= TOL_OUT, errs
     assert max(errs.values()) <= TOL_GRAD, errs
+
+
+def test_merged_weight_reproduces_the_forward():
+    """Export: the module's merged bf16 weight W' = W^ + s B A, used in a plain
+    product, gives the layer's forward (oracle, fp64) within the tolerance;
+    the same holds for an FP4 module."""
+    torch.cuda.set_device(0)
+    for codebook, name in ((B.QLORA_CODEBOOK_NF4, "nf4"), (B.QLORA_CODEBOOK_FP4, "fp4")):
+        case = WL.LinearCase("merge_module", n=520, k=640, m=96, r=16, alpha=32.0, w_seed=990, x_seed=991,
+                             a_seed=992, b_seed=993, dy_seed=994)
+        lin = L.QLoRALinear.from_float(case.W().to(DEV), case.A().to(DEV), case.B().to(DEV), case.alpha,
+                                       codebook=codebook)
+        assert lin.w.codebook == codebook
+        X = case.X().to(DEV)
+        Wm = lin.merged_weight()
+        Y2 = (X.double() @ Wm.double().t())
+        torch.cuda.synchronize()
+        ref = R.fwd(R.bf16_to_f64(case.X()), R.dequant_full(case.W(), name), R.bf16_to_f64(case.A()),
+                    R.bf16_to_f64(case.B()), case.scale)
+        assert R.err(Y2.cpu().numpy(), ref) <= TOL_OUT
+        assert lin.merged_weight(torch.float32).dtype == torch.float32
