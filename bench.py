@@ -312,6 +312,170 @@ def _m1_decode(dev, peaks, peak_kind):
     return out
 
 
+def _graph_time(calls, reps_bytes: int, bytes_per_call: int) -> float:
+    """Seconds per call of `calls` (a list of closures, one per rotating input
+    copy) replayed from one CUDA graph, after a warm-up outside capture."""
+    import torch
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for c in calls:
+            c()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for c in calls:
+                c()
+    reps = max(3, int(reps_bytes // max(1, bytes_per_call * len(calls))) + 1)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e-3 / (reps * len(calls))
+
+
+def _decode_small_m(dev, peaks, peak_kind):
+    """The 7B attention projection [4096 x 4096] (0.1 % outliers, r=16) at
+    M = 4 and 16: weight-GB/s over rotating weight copies larger than 2x L2,
+    replayed from a CUDA graph."""
+    import torch
+    from bit_nf4_quantized_qlora_b200 import binding as B
+    from bit_nf4_quantized_qlora_b200 import workloads as WL
+    out = {}
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    case = WL.attn_proj_7b(1)
+    wb = weight_bytes(case.n, case.k)
+    copies = max(2, int(2 * l2 // wb) + 1)
+    w0 = B.qlora_quantize_nf4_dq(case.W().to(dev))
+    ws = [w0] + [B.NF4Weight(w0.codes.clone(), w0.absmax_q.clone(), w0.group_scale.clone(), case.n, case.k)
+                 for _ in range(copies - 1)]
+    A, Bm = case.A().to(dev), case.B().to(dev)
+    for m in (4, 16):
+        X = case.X(m).to(dev)
+        Y = torch.empty(m, case.n, dtype=torch.bfloat16, device=dev)
+        wsp = torch.empty(B.qlora_workspace_bytes(B.QLORA_OP_FWD, m, case.n, case.k, case.r), dtype=torch.uint8,
+                          device=dev)
+        calls = [lambda w=w: B.qlora_linear_fwd(X, w, A, Bm, case.r, case.scale, out=Y, ws=wsp) for w in ws]
+        t = _graph_time(calls, 200e6, wb)
+        moved = wb + 2 * case.r * (case.n + case.k) + 2 * m * (case.n + case.k)
+        gbs = moved / t / 1e9
+        fl = linear_flops(m, case.n, case.k, case.r)["fwd"]
+        out[f"m{m}"] = {"us_per_call": round(t * 1e6, 3), "gbps": round(gbs, 1),
+                        "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4), "tflops": round(fl / t / 1e12, 2),
+                        "weight_copies": copies, "cuda_graph": True}
+    out["workload"] = "7B attention projection W [4096 x 4096] NF4 (0.1% outliers at 10 sigma), LoRA r=16"
+    out["peak_kind"] = peak_kind
+    out["bytes"] = "codes + absmax codes + group scales + A, B + X, Y per call"
+    del ws, w0
+    torch.cuda.empty_cache()
+    return out
+
+
+def _up_proj_70b_sweep(dev, peaks, peak_kind, reps: int = 5):
+    """70B up-projection W [28672 x 8192] (r=16, alpha=32) at M = 16, 128,
+    1024 and 8192: forward and input gradient, algorithmic TFLOP/s of each
+    call against the burst bf16 peak; at M = 16 and 128 also the HBM fraction
+    of the bytes one call must move (weight once, X, Y or dY, dX, adapters).
+    Two weight copies alternate so the weight is never read from L2 twice in
+    a row (121 MB each, with the activations, exceeds the 126 MB L2)."""
+    import torch
+    from bit_nf4_quantized_qlora_b200 import binding as B
+    from bit_nf4_quantized_qlora_b200 import workloads as WL
+    case = WL.up_proj_70b(1)
+    n, k, r = case.n, case.k, case.r
+    g = torch.Generator(device=dev)
+    g.manual_seed(31)
+    W = torch.randn(n, k, generator=g, device=dev, dtype=torch.float32) * case.w_std
+    w0 = B.qlora_quantize_nf4_dq(W)
+    del W
+    ws = [w0, B.NF4Weight(w0.codes.clone(), w0.absmax_q.clone(), w0.group_scale.clone(), n, k)]
+    A = (torch.randn(r, k, generator=g, device=dev) * 0.01).to(torch.bfloat16)
+    Bm = (torch.randn(n, r, generator=g, device=dev) * 0.01).to(torch.bfloat16)
+    wb = weight_bytes(n, k)
+    out = {}
+    for m in (16, 128, 1024, 8192):
+        X = torch.randn(m, k, generator=g, device=dev).to(torch.bfloat16)
+        dY = torch.randn(m, n, generator=g, device=dev).to(torch.bfloat16)
+        Y = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
+        dX = torch.empty(m, k, dtype=torch.bfloat16, device=dev)
+        wsf = torch.empty(max(1, B.qlora_workspace_bytes(B.QLORA_OP_FWD, m, n, k, r)), dtype=torch.uint8, device=dev)
+        wsb = torch.empty(max(1, B.qlora_workspace_bytes(B.QLORA_OP_BWD_DX, m, n, k, r)), dtype=torch.uint8,
+                          device=dev)
+        row = {}
+        for name, fn in (("fwd", lambda i: B.qlora_linear_fwd(X, ws[i % 2], A, Bm, r, case.scale, out=Y, ws=wsf)),
+                         ("bwd_dx", lambda i: B.qlora_linear_bwd_dx(dY, ws[i % 2], A, Bm, r, case.scale, out=dX,
+                                                                    ws=wsb))):
+            for i in range(3):
+                fn(i)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for i in range(reps):
+                fn(i)
+            e1.record()
+            torch.cuda.synchronize()
+            t = e0.elapsed_time(e1) * 1e-3 / reps
+            fl = linear_flops(m, n, k, r)[name]
+            moved = wb + 2 * r * (n + k) + 2 * m * (n + k)
+            ent = {"us": round(t * 1e6, 1), "tflops": round(fl / t / 1e12, 1),
+                   "frac_of_bf16_peak": round(fl / t / 1e12 / peaks["bf16_tflops"], 4)}
+            if m <= 128:
+                ent["gbps"] = round(moved / t / 1e9, 1)
+                ent["frac_of_hbm"] = round(moved / t / 1e9 / peaks["hbm_gbs"], 4)
+            row[name] = ent
+        out[f"m{m}"] = row
+        del X, dY, Y, dX, wsf, wsb
+        torch.cuda.empty_cache()
+    out["workload"] = "70B up-projection W [28672 x 8192] NF4, LoRA r=16 alpha=32; calls through the C ABI"
+    out["peak_kind"] = f"{peak_kind}: bf16 burst {peaks['bf16_tflops']} TFLOP/s, HBM {peaks['hbm_gbs']} GB/s"
+    del ws, w0
+    torch.cuda.empty_cache()
+    return out
+
+
+def _quantize_dequant_70b(dev, peaks, peak_kind, reps: int = 5):
+    """Standalone quantize (fp32 W -> codes, absmax codes, group scales) and
+    dequant (-> bf16 W^) of the 70B up-projection weight, 234,881,024
+    elements: algorithmic GB/s (4 B read + 0.5157 B written per weight;
+    0.5157 B read + 2 B written per weight) against the measured HBM copy
+    bandwidth.  Each call moves about 1 GB, far above the L2."""
+    import torch
+    from bit_nf4_quantized_qlora_b200 import binding as B
+    n, k = 28672, 8192
+    numel = n * k
+    g = torch.Generator(device=dev)
+    g.manual_seed(31)
+    W = torch.randn(n, k, generator=g, device=dev, dtype=torch.float32) * 0.015
+    w = B.qlora_quantize_nf4_dq(W)
+    Wd = torch.empty(n, k, dtype=torch.bfloat16, device=dev)
+    wb = weight_bytes(n, k)
+    out = {}
+    for name, fn, moved in (("quantize", lambda: B.qlora_quantize_nf4_dq(W, out=w), 4 * numel + wb),
+                            ("dequant", lambda: B.qlora_dequant(w, out=Wd), wb + 2 * numel)):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) * 1e-3 / reps
+        gbs = moved / t / 1e9
+        out[name] = {"us": round(t * 1e6, 1), "gbps": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                     "bytes_per_call": int(moved)}
+    out["workload"] = "70B up-projection weight [28672 x 8192] fp32 N(0, 0.015), NF4 block 64, DQ per 256 blocks"
+    out["peak_kind"] = peak_kind
+    del W, w, Wd
+    torch.cuda.empty_cache()
+    return out
+
+
 def _decoder_layer(dev, steps: int = 5, warmup: int = 2):
     """7B-shaped decoder block (q, k, v, o, gate, up, down all NF4 + LoRA
     r=64, attention/RMSNorm/SwiGLU in PyTorch), X [2 x 2048 x 4096]: device
@@ -547,18 +711,25 @@ def run_ours(args):
     t_launch = sum(gu) / len(gu)
     f_launch = linear_flops(cases[0].m, cases[0].n, cases[0].k, cases[0].r)["fused_fwd_kernel"]
     achieved = f_launch / t_launch / 1e12
-    peak = peaks["bf16_tflops_sustained"]
+    # The timed region is tens of milliseconds, far from the seconds-long
+    # power-capped loop of the sustained figure: the burst peak applies.
+    peak = peaks["bf16_tflops"]
     traffic = profile_traffic(kernel_source_digest())
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "kernel": "fused_fwd_kernel: NF4 dequant + tcgen05 GEMM (forward, 4096x11008x4096, LoRA r=64)",
                 "flops_per_launch": f_launch, "launch_us": round(t_launch * 1e6, 2),
-                "peak_kind": f"{peak_kind} sustained bf16 (cuBLAS, long loop under the power cap)"}
+                "peak_kind": f"{peak_kind} burst bf16 (cuBLAS 8192^3, best of 10)",
+                "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                "sustained_peak": peaks["bf16_tflops_sustained"]}
 
     # End to end through the public API with host buffers.
     e2e = _e2e(projs, cases, flat, world, dev, stream, max(3, min(K, 10)))
 
     m1 = _m1_decode(dev, peaks, peak_kind) if rank == 0 else None
+    decode_small = _decode_small_m(dev, peaks, peak_kind) if rank == 0 else None
+    sweep = _up_proj_70b_sweep(dev, peaks, peak_kind) if rank == 0 else None
+    qd = _quantize_dequant_70b(dev, peaks, peak_kind) if rank == 0 else None
     layer = _decoder_layer(dev) if rank == 0 else None
     unfused = _unfused_comparator(projs[0], dev) if rank == 0 else None
     codebook = _codebook_error(dev) if rank == 0 else None
@@ -581,6 +752,9 @@ def run_ours(args):
             "gpu_launches": int(launches),
             "clocks": clk.summary(),
             "m1_decode": m1,
+            "attn_proj_decode_m4_m16": decode_small,
+            "up_proj_70b_m_sweep": sweep,
+            "quantize_dequant_70b": qd,
             "decoder_layer_7b": layer,
             "unfused_comparator": unfused,
             "codebook_error": codebook,
@@ -627,7 +801,10 @@ def _e2e(projs, cases, flat, world, dev, stream, steps):
     el = reduce_max(t0.elapsed_time(t1) * 1e-3, world, dev)
     value = step_flops(cases) * world * steps / el / 1e12
     return {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "steps": steps, "ms_per_step": round(el / steps * 1e3, 3)}
+            "steps": steps, "ms_per_step": round(el / steps * 1e3, 3),
+            "scope": "per step: X and dY of the three projections copied in from pinned host memory, the "
+                     "adapter gradients copied out; Y and dX stay on the device (activations of a training "
+                     "step are consumed there)"}
 
 
 # ---------------------------------------------------------------------------

@@ -31,6 +31,14 @@ QLORA_CODEBOOK_FP4 = 1
 QLORA_CODEBOOK_INT4 = 2
 CODEBOOKS = {"nf4": QLORA_CODEBOOK_NF4, "fp4": QLORA_CODEBOOK_FP4, "int4": QLORA_CODEBOOK_INT4}
 
+# Bits of the device error word (qlora_poll_device_error).
+QLORA_DEVERR_OPERANDS = 1 << 0
+QLORA_DEVERR_WEIGHT_TILE = 1 << 1
+QLORA_DEVERR_FREE_STAGE = 1 << 2
+QLORA_DEVERR_ACCUMULATOR = 1 << 3
+QLORA_DEVERR_DRAIN = 1 << 4
+QLORA_DEVERR_SELFTEST = 1 << 5
+
 QLORA_OP_FWD = 0
 QLORA_OP_BWD_DX = 1
 QLORA_OP_LORA_BWD = 2
@@ -90,6 +98,8 @@ _SIGNATURES = {
     "qlora_linear_fwd_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(NF4WeightC),
                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_float,
                                                 ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_selftest_div255": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_uint32, ctypes.c_void_p, ctypes.c_void_p]),
 }
 
 
@@ -327,3 +337,21 @@ def qlora_linear_fwd_noalloc(X: torch.Tensor, w: NF4Weight, A: Optional[torch.Te
            lib().qlora_linear_fwd_noalloc(X.data_ptr(), m, ctypes.byref(ws_c), _ptr(A), _ptr(B), r, float(scale),
                                           out.data_ptr(), _stream(stream)))
     return out
+
+
+def qlora_selftest_bounded_wait(limit_ns: int, expired: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Launch the bounded-wait self-test (a wait on a barrier nothing arrives
+    at, given up after limit_ns); `expired` is an int32 [1] device tensor that
+    receives 1 when the wait ran out."""
+    _need_cuda(expired)
+    _check("qlora_selftest_bounded_wait",
+           lib().qlora_selftest_bounded_wait(int(limit_ns), _ptr(expired), _stream(stream)))
+
+
+def qlora_selftest_div255(first_bits: int, count: int, mismatches: torch.Tensor, stream=None) -> None:
+    """Add to the int64 [1] device tensor `mismatches` the number of fp32 bit
+    patterns in [first_bits, first_bits + count) whose library fp32(s / 255)
+    differs from IEEE division."""
+    _need_cuda(mismatches)
+    _check("qlora_selftest_div255",
+           lib().qlora_selftest_div255(int(first_bits), int(count), mismatches.data_ptr(), _stream(stream)))

@@ -37,27 +37,6 @@ int cuda_status(cudaError_t e) {
 
 size_t round_up(size_t v) { return (v + kWsAlign - 1) / kWsAlign * kWsAlign; }
 
-// The device the calls run on must be sm_100.  The first call on a host
-// thread also makes sure the runtime has a context current on that thread
-// (a thread that never touched CUDA, such as a framework's worker thread, may
-// have none yet; kernel configuration calls made before it is bound have
-// failed with cudaErrorInvalidValue).
-int check_device() {
-  thread_local int t_ready_dev = -1;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_status(e);
-  if (t_ready_dev != dev) {
-    e = cudaFree(nullptr);
-    if (e != cudaSuccess) return cuda_status(e);
-    t_ready_dev = dev;
-  }
-  int major = 0;
-  e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-  if (e != cudaSuccess) return cuda_status(e);
-  return major == 10 ? QLORA_OK : QLORA_ERR_DEVICE;
-}
-
 // The linear operations also need n % 8 == 0 (16-byte rows of Y and dY).
 int check_weight(const qlora_nf4_weight *w, bool linear = true) {
   if (!w || !w->codes || !w->absmax_q || !w->group_scale) return QLORA_ERR_NULL;
@@ -85,21 +64,104 @@ WeightView view(const qlora_nf4_weight *w) {
   return WeightView{w->codes, w->absmax_q, w->group_scale, w->n, w->k, &codebook_tables(w->codebook)};
 }
 
+constexpr int kMaxDevices = kMaxDevicesPerProcess;
+
 }  // namespace
+
+// The device the calls run on must be sm_100.  The first call on a host
+// thread also makes sure the runtime has a context current on that thread
+// (a thread that never touched CUDA, such as a framework's worker thread, may
+// have none yet; kernel configuration calls made before it is bound have
+// failed with cudaErrorInvalidValue).  cudaSetDevice binds the device's
+// primary context to the calling thread and allocates nothing.
+int check_device() {
+  thread_local int t_ready_dev = -1;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (t_ready_dev != dev) {
+    e = cudaSetDevice(dev);
+    if (e != cudaSuccess) return cuda_status(e);
+    t_ready_dev = dev;
+  }
+  int major = 0;
+  e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  return major == 10 ? QLORA_OK : QLORA_ERR_DEVICE;
+}
 
 int status_from_cuda(cudaError_t e) { return cuda_status(e); }
 
 void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
+// The error word's device address, looked up once per device.  Two threads
+// on a fresh device may both look it up; they store the same value, and the
+// slots are atomics, so the race is harmless.
 unsigned *device_error_word() {
-  static unsigned *cache[64] = {};
+  static std::atomic<unsigned *> cache[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-  if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+  const bool slot = dev >= 0 && dev < kMaxDevices;
+  if (slot) {
+    unsigned *p = cache[dev].load(std::memory_order_acquire);
+    if (p) return p;
+  }
   void *ptr = nullptr;
   if (cudaGetSymbolAddress(&ptr, g_device_error) != cudaSuccess) return nullptr;
-  if (dev >= 0 && dev < 64) cache[dev] = static_cast<unsigned *>(ptr);
+  if (slot) cache[dev].store(static_cast<unsigned *>(ptr), std::memory_order_release);
   return static_cast<unsigned *>(ptr);
+}
+
+cudaError_t set_smem_once(const void *kernel, int smem_bytes, std::atomic<bool> *done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool slot = dev >= 0 && dev < kMaxDevices;
+  if (slot && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  if (e == cudaSuccess && slot) done[dev].store(true, std::memory_order_release);
+  return e;
+}
+
+int validate_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w, const uint16_t *A, const uint16_t *B,
+                 int32_t r, uint16_t *Y, bool *use_adapter) {
+  int st = check_weight(w);
+  if (st != QLORA_OK) return st;
+  st = check_adapter(A, B, r, use_adapter);
+  if (st != QLORA_OK) return st;
+  if (m < 0 || m > (int64_t(1) << 31)) return QLORA_ERR_SHAPE;
+  if (m == 0) return QLORA_OK;
+  if (!X || !Y) return QLORA_ERR_NULL;
+  if (!aligned16(X) || !aligned16(Y)) return QLORA_ERR_ALIGN;
+  return QLORA_OK;
+}
+
+int launch_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w, const uint16_t *A, const uint16_t *B,
+               int32_t r, float scale, uint16_t *Y, uint16_t *T, cudaStream_t s) {
+  const bool lora = T != nullptr;
+  cudaError_t e = cudaSuccess;
+  // The main kernel overlaps the adapter projection (programmatic dependent
+  // launch) unless the caller is timing the main kernel alone.
+  const bool pdl = lora && t_prof_start == nullptr;
+  if (m <= kSmallM) {
+    if (lora) e = launch_lora_proj_small(X, m, w->k, A, r, scale, T, s);
+    if (e == cudaSuccess) e = prof_mark(t_prof_start, s);
+    if (e == cudaSuccess) {
+      // Decode sizes take the per-warp streaming kernel; the rest (m > 4,
+      // or K beyond one cluster's warps) the CTA-ring kernel.
+      e = gemv_stream_supported(m, w->n, w->k)
+              ? launch_gemv_stream(X, m, w->codes, w->absmax_q, w->group_scale, w->n, w->k, T,
+                                   lora ? B : nullptr, lora ? r : 0, Y, codebook_tables(w->codebook), s, pdl)
+              : launch_gemv_fwd(X, m, w->codes, w->absmax_q, w->group_scale, w->n, w->k, T, lora ? B : nullptr,
+                                lora ? r : 0, Y, codebook_tables(w->codebook), s, pdl);
+    }
+  } else {
+    if (lora) e = tc_proj_kmajor(X, m, w->k, A, r, scale, T, s);
+    if (e == cudaSuccess) e = prof_mark(t_prof_start, s);
+    if (e == cudaSuccess) e = tc_fwd(X, m, view(w), T, lora ? B : nullptr, lora ? r : 0, Y, s, pdl);
+  }
+  if (e == cudaSuccess) e = prof_mark(t_prof_stop, s);
+  return cuda_status(e);
 }
 
 }  // namespace qlora
@@ -207,46 +269,16 @@ int qlora_dequant(const qlora_nf4_weight *w, uint16_t *W_bf16, qlora_stream_t st
 int qlora_linear_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w, const uint16_t *A,
                      const uint16_t *B, int32_t r, float scale, uint16_t *Y, void *ws, size_t ws_bytes,
                      qlora_stream_t stream) {
-  int st = check_weight(w);
-  if (st != QLORA_OK) return st;
   bool lora = false;
-  st = check_adapter(A, B, r, &lora);
-  if (st != QLORA_OK) return st;
-  if (m < 0 || m > (int64_t(1) << 31)) return QLORA_ERR_SHAPE;
-  if (m == 0) return QLORA_OK;
-  if (!X || !Y) return QLORA_ERR_NULL;
-  if (!aligned16(X) || !aligned16(Y)) return QLORA_ERR_ALIGN;
+  int st = validate_fwd(X, m, w, A, B, r, Y, &lora);
+  if (st != QLORA_OK || m == 0) return st;
   const size_t need = lora ? qlora_workspace_bytes(QLORA_OP_FWD, m, w->n, w->k, r) : 0;
   if (need > 0 && (ws == nullptr || ws_bytes < need)) return QLORA_ERR_WORKSPACE;
   if (ws && !aligned16(ws)) return QLORA_ERR_ALIGN;
   st = check_device();
   if (st != QLORA_OK) return st;
-
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  uint16_t *T = lora ? static_cast<uint16_t *>(ws) : nullptr;
-  cudaError_t e = cudaSuccess;
-  // The main kernel overlaps the adapter projection (programmatic dependent
-  // launch) unless the caller is timing the main kernel alone.
-  const bool pdl = lora && t_prof_start == nullptr;
-  if (m <= kSmallM) {
-    if (lora) e = launch_lora_proj_small(X, m, w->k, A, r, scale, T, s);
-    if (e == cudaSuccess) e = prof_mark(t_prof_start, s);
-    if (e == cudaSuccess) {
-      // Decode sizes take the per-warp streaming kernel; the rest (m > 4,
-      // or K beyond one cluster's warps) the CTA-ring kernel.
-      e = gemv_stream_supported(m, w->n, w->k)
-              ? launch_gemv_stream(X, m, w->codes, w->absmax_q, w->group_scale, w->n, w->k, T,
-                                   lora ? B : nullptr, lora ? r : 0, Y, codebook_tables(w->codebook), s, pdl)
-              : launch_gemv_fwd(X, m, w->codes, w->absmax_q, w->group_scale, w->n, w->k, T, lora ? B : nullptr,
-                                lora ? r : 0, Y, codebook_tables(w->codebook), s, pdl);
-    }
-  } else {
-    if (lora) e = tc_proj_kmajor(X, m, w->k, A, r, scale, T, s);
-    if (e == cudaSuccess) e = prof_mark(t_prof_start, s);
-    if (e == cudaSuccess) e = tc_fwd(X, m, view(w), T, lora ? B : nullptr, lora ? r : 0, Y, s, pdl);
-  }
-  if (e == cudaSuccess) e = prof_mark(t_prof_stop, s);
-  return cuda_status(e);
+  return launch_fwd(X, m, w, A, B, r, scale, Y, lora ? static_cast<uint16_t *>(ws) : nullptr,
+                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 int qlora_linear_bwd_dx(const uint16_t *dY, int64_t m, const qlora_nf4_weight *w, const uint16_t *A,

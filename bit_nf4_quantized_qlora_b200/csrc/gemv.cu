@@ -401,16 +401,15 @@ cudaError_t launch_gemv_fwd(const uint16_t *X, int64_t m, const uint8_t *codes, 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  static bool configured[64][2] = {};
+  static std::atomic<bool> configured1[kMaxDevicesPerProcess] = {}, configured2[kMaxDevicesPerProcess] = {};
   const int variant = m <= 8 ? 0 : 1;
-  if (dev >= 0 && dev < 64 && !configured[dev][variant]) {
-    cudaError_t e = variant == 0
-                        ? cudaFuncSetAttribute(gemv_fwd_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(kSmemBytes))
-                        : cudaFuncSetAttribute(gemv_fwd_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(kSmemBytes));
+  {
+    const cudaError_t e =
+        variant == 0 ? set_smem_once(reinterpret_cast<const void *>(gemv_fwd_kernel<1>), static_cast<int>(kSmemBytes),
+                                     configured1)
+                     : set_smem_once(reinterpret_cast<const void *>(gemv_fwd_kernel<2>), static_cast<int>(kSmemBytes),
+                                     configured2);
     if (e != cudaSuccess) return e;
-    configured[dev][variant] = true;
   }
   // Split K over a cluster of cs CTAs.  Pick cs in 1..8 to fill the resident
   // CTA slots (two per SM) in as few, as full waves as possible, keeping at

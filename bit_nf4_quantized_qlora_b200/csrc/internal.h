@@ -1,14 +1,19 @@
 // Host-side declarations shared by the translation units of libqlora.
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "../../include/qlora.h"
 #include "types.h"
 
 namespace qlora {
+
+// Per-device tables of the library (attribute flags, cached addresses).
+constexpr int kMaxDevicesPerProcess = 64;
 
 // The library's codebooks and their midpoints (derived once at load time):
 // codebook_tables(kCodebookNF4 | kCodebookFP4 | kCodebookINT4).
@@ -24,6 +29,27 @@ void count_launches(int n);
 // QLORA_OK for cudaSuccess; otherwise records the error for
 // qlora_last_cuda_error() and returns QLORA_ERR_CUDA.
 int status_from_cuda(cudaError_t e);
+
+// QLORA_OK when the current device is an sm_100 part (binding the device's
+// primary context to this thread on its first call); QLORA_ERR_DEVICE or
+// QLORA_ERR_CUDA otherwise.
+int check_device();
+
+// Raises a kernel's dynamic shared-memory limit once per device (`done`
+// holds one flag per device; the attribute call is idempotent, so two threads
+// that race on a fresh device both set the same value).
+cudaError_t set_smem_once(const void *kernel, int smem_bytes, std::atomic<bool> *done);
+
+// Host-side checks of a forward call (weight, adapter, m, X, Y), in the order
+// every forward entry point reports them; *use_adapter tells whether the call
+// has an adapter.  No CUDA call is made.
+int validate_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w, const uint16_t *A, const uint16_t *B,
+                 int32_t r, uint16_t *Y, bool *use_adapter);
+
+// Launches a validated forward (m > 0) with T as the rank-r scratch (null:
+// no adapter); returns a qlora status.
+int launch_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w, const uint16_t *A, const uint16_t *B,
+               int32_t r, float scale, uint16_t *Y, uint16_t *T, cudaStream_t s);
 
 // TMA tensor maps (2D, row-major).  bf16: 128-byte swizzle.  codes: uint8
 // rows of packed codes, optional 128-byte swizzle.  False if encoding failed.

@@ -245,12 +245,11 @@ cudaError_t launch_merge(const WeightView &w, const uint16_t *A, const uint16_t 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  static uint32_t configured[64] = {};
-  if (dev >= 0 && dev < 64 && configured[dev] < smem) {
-    e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    configured[dev] = smem;
-  }
+  // The limit is raised once per device to what the largest rank needs, so
+  // concurrent calls with different ranks never lower it under one another.
+  static std::atomic<bool> configured[kMaxDevicesPerProcess] = {};
+  e = set_smem_once(reinterpret_cast<const void *>(merge_kernel), static_cast<int>(Layout(256).total), configured);
+  if (e != cudaSuccess) return e;
   const dim3 grid(static_cast<unsigned>((w.k + kTN - 1) / kTN), static_cast<unsigned>((w.n + kTM - 1) / kTM), 1);
   merge_kernel<<<grid, kThreads, smem, stream>>>(p);
   count_launches(1);

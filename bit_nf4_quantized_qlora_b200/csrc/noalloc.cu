@@ -23,28 +23,53 @@ constexpr size_t kNoallocScratchBytes = QLORA_NOALLOC_SCRATCH_BYTES;
 // Every device that loads the library holds this array until process exit.
 static __device__ __align__(256) unsigned char g_fwd_scratch[kNoallocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void *g_scratch_ptr[kMaxDevices] = {};
+// The driver context current on this thread (null if none, or if the driver
+// entry point is unavailable), fetched through the runtime so that the
+// library does not link libcuda.
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
 
-// The array's device address for the current device.  In host code the
-// symbol itself is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetCurrentFn>(f);
+    return static_cast<CtxGetCurrentFn>(nullptr);
+  }();
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// The array's device address as seen from the context that is current now.
+// In host code the symbol itself is only a host-side stand-in, so the address
+// is looked up with the device current (cudaGetSymbolAddress) the first time a
+// device is used, and again whenever a different driver context is current on
+// that device (each context loads its own copy of the library's module).
+struct ScratchSlot {
+  CUcontext ctx = nullptr;
+  void *ptr = nullptr;
+};
+std::mutex g_scratch_mutex;
+ScratchSlot g_scratch[kMaxDevicesPerProcess];
+
 cudaError_t scratch_address(void **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= kMaxDevicesPerProcess) return cudaErrorInvalidDevice;
+  const CUcontext ctx = current_context();
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  ScratchSlot &s = g_scratch[dev];
+  if (s.ptr == nullptr || s.ctx != ctx) {
     void *p = nullptr;
-    e = cudaFree(nullptr);   // a context current on this thread before the lookup
-    if (e != cudaSuccess) return e;
     e = cudaGetSymbolAddress(&p, g_fwd_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
+    s.ptr = p;
+    s.ctx = ctx;
   }
-  *out = g_scratch_ptr[dev];
+  *out = s.ptr;
   return cudaSuccess;
 }
 
@@ -54,18 +79,20 @@ cudaError_t scratch_address(void **out) {
 extern "C" int qlora_linear_fwd_noalloc(const uint16_t *X, int64_t m, const qlora_nf4_weight *w,
                                         const uint16_t *A, const uint16_t *B, int32_t r, float scale,
                                         uint16_t *Y, qlora_stream_t stream) {
-  if (!w) return QLORA_ERR_NULL;
+  // The same checks, in the same order, as qlora_linear_fwd; the built-in
+  // scratch then stands where the caller's workspace would be checked.
+  bool lora = false;
+  int st = qlora::validate_fwd(X, m, w, A, B, r, Y, &lora);
+  if (st != QLORA_OK || m == 0) return st;
   void *scratch = nullptr;
-  size_t cap = 0;
-  const bool lora = r > 0 && (A != nullptr || B != nullptr);
-  // Only a well-formed adapter call needs the scratch; everything else is
-  // validated (and rejected) by qlora_linear_fwd exactly as for any caller.
-  if (lora && m > 0 && (r % 16) == 0 && r <= 256 && w->n > 0 && w->k > 0) {
-    const size_t need = qlora_workspace_bytes(QLORA_OP_FWD, m, w->n, w->k, r);
-    if (need > qlora::kNoallocScratchBytes) return QLORA_ERR_WORKSPACE;
+  if (lora && qlora_workspace_bytes(QLORA_OP_FWD, m, w->n, w->k, r) > qlora::kNoallocScratchBytes)
+    return QLORA_ERR_WORKSPACE;
+  st = qlora::check_device();
+  if (st != QLORA_OK) return st;
+  if (lora) {
     const cudaError_t e = qlora::scratch_address(&scratch);
     if (e != cudaSuccess) return qlora::status_from_cuda(e);
-    cap = qlora::kNoallocScratchBytes;
   }
-  return qlora_linear_fwd(X, m, w, A, B, r, scale, Y, scratch, cap, stream);
+  return qlora::launch_fwd(X, m, w, A, B, r, scale, Y, static_cast<uint16_t *>(scratch),
+                           reinterpret_cast<cudaStream_t>(stream));
 }

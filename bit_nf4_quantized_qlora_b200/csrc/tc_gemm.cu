@@ -445,16 +445,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
 template <class C>
 cudaError_t launch(const TcParams &p, int grid_n, int grid_m, cudaStream_t stream, int split = 1,
                    bool pdl = false) {
-  static bool configured[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static std::atomic<bool> configured[kMaxDevicesPerProcess] = {};
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(tc_kernel<C>), static_cast<int>(C::SMEM_BYTES),
+                                configured);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || !configured[dev]) {
-    e = cudaFuncSetAttribute(tc_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(C::SMEM_BYTES));
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) configured[dev] = true;
-  }
   if (grid_n <= 0 || grid_m <= 0) return cudaSuccess;
   if (split < 1 || !C::SPLIT) split = 1;
   cudaLaunchConfig_t cfg{};

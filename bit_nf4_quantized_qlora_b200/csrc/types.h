@@ -25,6 +25,7 @@ enum : unsigned {
   kErrTimeoutEmpty = 1u << 2,
   kErrTimeoutAcc = 1u << 3,
   kErrTimeoutDrain = 1u << 4,
+  kErrTimeoutSelfTest = 1u << 5,
 };
 
 }  // namespace qlora

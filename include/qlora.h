@@ -211,7 +211,8 @@ int qlora_lora_bwd(const uint16_t *X, const uint16_t *dY, int64_t m, int64_t n, 
  * deployment that forbids allocation on its serving path, or a C caller with
  * no device allocator.  The pages have no counterpart: this is a convenience
  * of this library around qlora_linear_fwd.
- *   Same arguments, semantics and results as qlora_linear_fwd, minus `ws`.
+ *   Same arguments, checks (in the same order), results and errors as
+ *   qlora_linear_fwd, minus `ws`.
  *   The rank-r scratch T lives in a fixed device array of
  *   QLORA_NOALLOC_SCRATCH_BYTES inside the library; every device that loads
  *   the library holds it until the process exits.  Calls whose scratch
@@ -219,8 +220,10 @@ int qlora_lora_bwd(const uint16_t *X, const uint16_t *dY, int64_t m, int64_t n, 
  *   launch nothing.  The call allocates nothing: no cudaMalloc, no cudaFree,
  *   no allocating library routine.
  *   The first call with an adapter on a device looks up the array's device
- *   address (cudaGetSymbolAddress) with that device current; make that first
- *   call before any stream capture.
+ *   address (cudaGetSymbolAddress) with that device current, and looks it up
+ *   again whenever another driver context is current on that device; make
+ *   that first call before any stream capture.  Calls after cudaDeviceReset
+ *   in the same process are not supported.
  *   All calls on a device share the array and it keeps the last call's
  *   contents; T is fully written before it is read, so nothing in it needs to
  *   start at zero.  Calls that may run at the same time on one device (other
@@ -242,8 +245,34 @@ int qlora_last_cuda_error(void);
  * up after its time limit sets a bit in a per-device error word instead and
  * the kernel exits early (its outputs are then undefined).  This call
  * synchronizes `stream`, writes the word to *flags (host memory; 0 = no
- * error) and clears it.  QLORA_ERR_NULL if flags is NULL.                   */
+ * error) and clears it.  QLORA_ERR_NULL if flags is NULL.  Bits: which wait
+ * gave up (a pipeline stage's operands, the expanded weight tile, a free
+ * stage, the accumulator, the final drain of copies, the self-test).        */
+enum qlora_device_error {
+  QLORA_DEVERR_OPERANDS = 1u << 0,
+  QLORA_DEVERR_WEIGHT_TILE = 1u << 1,
+  QLORA_DEVERR_FREE_STAGE = 1u << 2,
+  QLORA_DEVERR_ACCUMULATOR = 1u << 3,
+  QLORA_DEVERR_DRAIN = 1u << 4,
+  QLORA_DEVERR_SELFTEST = 1u << 5
+};
 int qlora_poll_device_error(qlora_stream_t stream, unsigned *flags);
+
+/* Self-tests of the device-side guards (no counterpart on the pages).
+ * qlora_selftest_bounded_wait launches one thread that waits, through the
+ * same bounded mbarrier wait the pipelined kernels use, on a barrier nothing
+ * arrives at: after limit_ns nanoseconds (1 .. 2e9) the wait gives up, sets
+ * QLORA_DEVERR_SELFTEST in the device error word and the kernel returns,
+ * writing 1 to *expired (device memory, 4-byte aligned; may be NULL).  Nothing
+ * faults and the context stays usable.
+ * qlora_selftest_div255 adds to *mismatches (device memory, 8-byte aligned)
+ * the number of fp32 bit patterns in [first_bits, first_bits + count) (all
+ * positive and finite) whose fp32(s / 255) by the library's division
+ * (Markstein's method with the correctly rounded reciprocal of 255, used for
+ * the double-quantization constant) differs from IEEE division.             */
+int qlora_selftest_bounded_wait(uint64_t limit_ns, unsigned *expired, qlora_stream_t stream);
+int qlora_selftest_div255(uint32_t first_bits, uint32_t count, unsigned long long *mismatches,
+                          qlora_stream_t stream);
 
 /* Profiling hook.  While set, qlora_linear_fwd and qlora_linear_bwd_dx
  * record `start` on their stream right before launching their main kernel

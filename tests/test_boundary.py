@@ -203,3 +203,40 @@ def test_quantize_and_dequant_reject_bad_arguments(lib):
 
 def test_poll_rejects_null(lib):
     assert lib.qlora_poll_device_error(None, None) == B.QLORA_ERR_NULL
+
+
+def _noalloc(lib, X=P, m=16, w=None, A=P, Bm=P, r=16, Y=P):
+    w = w if w is not None else _w()
+    return lib.qlora_linear_fwd_noalloc(X, m, ctypes.byref(w), A, Bm, r, 2.0, Y, None)
+
+
+def test_noalloc_reports_errors_in_the_order_of_the_workspace_forward(lib):
+    """Every host-side check of the forward comes before the built-in
+    scratch's size check, so a bad weight or a half adapter is reported as
+    such even when m is too large for the scratch."""
+    big = (1 << 20) // (2 * 256) + 1                                 # m * r * 2 beyond the scratch at r = 256
+    assert _noalloc(lib, m=big, r=256, w=_w(k=1000)) == B.QLORA_ERR_SHAPE
+    assert _noalloc(lib, m=big, r=256, A=None) == B.QLORA_ERR_NULL
+    assert _noalloc(lib, m=big, r=256, w=_w(codes=0)) == B.QLORA_ERR_NULL
+    assert _noalloc(lib, m=big, r=256, X=MIS) == B.QLORA_ERR_ALIGN
+    assert _noalloc(lib, m=big, r=256) == B.QLORA_ERR_WORKSPACE
+    for kw in (dict(X=None), dict(Y=MIS), dict(w=_w(n=1020)), dict(r=12), dict(m=-1), dict(A=MIS)):
+        assert _noalloc(lib, **kw) == _fwd(lib, **kw), kw
+    assert _noalloc(lib, m=0, X=None, Y=None) == B.QLORA_OK
+
+
+def test_selftests_reject_bad_arguments(lib):
+    assert lib.qlora_selftest_bounded_wait(0, None, None) == B.QLORA_ERR_SHAPE
+    assert lib.qlora_selftest_bounded_wait(3_000_000_000, None, None) == B.QLORA_ERR_SHAPE
+    assert lib.qlora_selftest_bounded_wait(1000, MIS + 1, None) == B.QLORA_ERR_ALIGN
+    assert lib.qlora_selftest_div255(0x3F800000, 16, None, None) == B.QLORA_ERR_NULL
+    assert lib.qlora_selftest_div255(0x3F800000, 16, P + 4, None) == B.QLORA_ERR_ALIGN
+    assert lib.qlora_selftest_div255(0x3F800000, 0, P, None) == B.QLORA_ERR_SHAPE
+    assert lib.qlora_selftest_div255(0x7F7FFFFF, 2, P, None) == B.QLORA_ERR_SHAPE    # would reach +inf
+
+
+def test_device_error_bits_match_the_header():
+    text = open(os.path.join(HEADER_DIR, "qlora.h")).read()
+    for name in ("OPERANDS", "WEIGHT_TILE", "FREE_STAGE", "ACCUMULATOR", "DRAIN", "SELFTEST"):
+        m = re.search(r"QLORA_DEVERR_%s\s*=\s*1u\s*<<\s*(\d+)" % name, text)
+        assert m and getattr(B, "QLORA_DEVERR_" + name) == 1 << int(m.group(1)), name
