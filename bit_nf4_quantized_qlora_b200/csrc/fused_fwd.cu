@@ -1,5 +1,7 @@
-// Fused NF4 forward for large M: Y = bf16(X . W^T + T . B^T), one 256 x 256
-// output tile per CTA, tcgen05 MMAs with the fp32 accumulator in TMEM.
+// Fused NF4 forward for large M: Y = bf16(X . W^T + T . B^T), computed by CTA
+// pairs.  Each pair of CTAs (a cluster of two) owns a 512 x 256 output tile;
+// its MMAs are tcgen05 pair MMAs (M = 256 over the two CTAs, N = 256) with the
+// fp32 accumulators in the two CTAs' tensor memory.
 //
 // "QLoRA and Quantized Training", The idea: each block is dequantized, used in
 // the multiply and discarded; "A 65B fine-tune on the GPU you already have",
@@ -7,21 +9,32 @@
 // exists in bf16 only as a 128-byte-swizzled shared-memory tile that dequant
 // warps write and the MMA reads.
 //
-// Rings and roles:
-//   stage ring (3 x 64 KB)  X tile [256 x 64] by TMA (the adapter T tile on
-//                           the extra k-steps) + the bf16 weight tile [256 x 64]
-//                           written by the dequant warps (the adapter's B tile,
-//                           on the extra k-steps, by plain loads)
-//   code rings (2 x 2 x 8 KB) packed codes [256 rows x 32 B] of a k-step, one
-//                           ring per dequant group
-//   warp 0 producer (X and code copies), warp 1 TMEM allocation + MMA issuer,
-//   warps 2..17 two groups of 8 dequant warps taking k-steps in turn (thread =
-//   one weight row = one NF4 block per k-step), then the epilogue.
-// The producer issues a k-step's codes only after the stage that step will use
-// has been released by the MMAs, so a group that sees its codes arrive knows
-// its weight slot is free.  Every barrier is waited on by its consumers use
-// after use (each group waits only on its own code ring), so a parity wait
-// can never be satisfied by an older phase.  Every wait is bounded in time (a
+// Why pairs: a pair MMA reads the N columns of its B operand half from each
+// CTA, so each CTA expands only 128 of the tile's 256 weight rows per k-step
+// while its tensor core still does the work of a 256 x 256 x 64 step.  That
+// halves the dequant instructions per FLOP and the shared-memory bytes the
+// tensor core reads per FLOP against a one-CTA tile of the same size.
+//
+// Per CTA (rank c of the pair; rows m0 = 512 p + 256 c of X, weight rows
+// n0 + 128 c .. + 128 of the pair's tile n0):
+//   stage ring, 4 x 52 KB  X rows [256 x 64] as two 128-row TMA boxes (the
+//                          adapter T on the extra k-steps), the bf16 weight
+//                          tile [128 x 64] (dequant warps; the adapter's B
+//                          rows by TMA on the extra k-steps) and the packed
+//                          codes [128 rows x 32 B] of the k-step
+//   warp 0   producer: X / T boxes with pair TMA counted on the leader's
+//            xfull barrier, codes with a local TMA on this CTA's cfull
+//   warp 1   tensor-memory allocation (both CTAs, 512 columns); in the
+//            leader CTA also the single thread that issues the pair MMAs
+//   warps 2..17  four groups of four dequant warps; group g expands the
+//            k-steps of stage g (one weight row = one NF4 block per thread)
+//            and arrives on the leader's wfull barrier; then the epilogue.
+// Barriers per stage: xfull (leader; X bytes of both CTAs), cfull (each CTA;
+// its codes), wfull (leader; 8 arrivals, the 4 + 4 dequant warps), empty
+// (each CTA; one arrival from the leader's multicast commit when the stage's
+// MMAs are done).  Every barrier is waited on by each of its waiters at every
+// phase (with four stages and four groups, group g owns stage g), so no parity
+// wait can be satisfied by an older phase.  Every wait is bounded in time (a
 // flag in the device error word on expiry); no kernel traps.
 #include "common.cuh"
 #include "internal.h"
@@ -30,26 +43,31 @@
 namespace qlora {
 namespace {
 
-constexpr int kBM = 256, kBN = 256, kBK = 64;
-constexpr int kStages = 3;
-constexpr int kGroups = 2, kGroupWarps = 8, kCodeSlots = 2;   // per group
-constexpr uint32_t kASub = 128u * kBK * 2u;          // one 128-row A sub-tile (16 KB)
+constexpr int kRowsCta = 256;                   // X rows per CTA (two 128-row MMA halves)
+constexpr int kBN = 256;                        // weight rows per pair tile
+constexpr int kWRows = kBN / 2;                 // weight rows expanded per CTA
+constexpr int kBK = 64;
+constexpr int kStages = 4;
+constexpr int kGroups = 4, kGroupWarps = 4;     // dequant: group g owns stage g
+constexpr uint32_t kASub = 128u * kBK * 2u;     // 16 KB: 128 X rows of a k-step
 constexpr uint32_t kABytes = 2u * kASub;
-constexpr uint32_t kBBytes = static_cast<uint32_t>(kBN) * kBK * 2u;
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr uint32_t kCBytes = static_cast<uint32_t>(kBN) * 32u;
-constexpr uint32_t kCOff = kStages * kStageBytes;
-constexpr uint32_t kSmemBytes = kCOff + kGroups * kCodeSlots * kCBytes + 1024u;
+constexpr uint32_t kBBytes = static_cast<uint32_t>(kWRows) * kBK * 2u;   // 16 KB
+constexpr uint32_t kCBytes = static_cast<uint32_t>(kWRows) * 32u;        // 4 KB
+constexpr uint32_t kBOff = kABytes, kCOff = kABytes + kBBytes;
+constexpr uint32_t kStageBytes = kABytes + kBBytes + kCBytes;            // 52 KB
+constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024u;
 constexpr int kThreads = 32 * (2 + kGroups * kGroupWarps);
-constexpr uint32_t kTmemCols = 512;                   // two 128 x 256 fp32 accumulators
-constexpr uint32_t kIdesc = make_idesc(kBN, false, false);
+constexpr uint32_t kTmemCols = 512;             // two 128 x 256 fp32 accumulators per CTA
+constexpr uint32_t kIdesc = make_idesc(kBN, false, false, 256);
+static_assert(kStages == kGroups, "each dequant group owns one stage");
+static_assert(kStageBytes % 1024u == 0, "1024-byte aligned operand tiles");
 static_assert(kSmemBytes <= 227u * 1024u, "shared memory");
 
 struct __align__(64) FwdParams {
   CUtensorMap tmA;       // X [m x k] bf16, box {64, 128}, 128B swizzle
-  CUtensorMap tmCodes;   // codes [n x k/2] bytes, box {32, 256}
+  CUtensorMap tmCodes;   // codes [n x k/2] bytes, box {32, 128}
   CUtensorMap tmA2;      // T [m x r] bf16, box {64, 128}, 128B swizzle
-  const uint16_t *B2;    // adapter B [n x r] bf16
+  CUtensorMap tmB2;      // adapter B [n x r] bf16, box {64, 128}, 128B swizzle
   const uint8_t *absmax_q;
   const float *group_scale;
   uint16_t *out;         // Y [m x n]
@@ -63,40 +81,42 @@ struct __align__(64) FwdParams {
 
 __global__ void __launch_bounds__(kThreads, 1) fused_fwd_kernel(const __grid_constant__ FwdParams p) {
   extern __shared__ uint8_t dsmem[];
-  __shared__ __align__(8) uint64_t full_a[kStages], full_b[kStages], empty[kStages];
-  __shared__ __align__(8) uint64_t c_full[kGroups][kCodeSlots], c_empty[kGroups][kCodeSlots];
-  __shared__ __align__(8) uint64_t acc_bar;
+  __shared__ __align__(8) uint64_t xfull[kStages], cfull[kStages], wfull[kStages], empty[kStages];
+  __shared__ __align__(8) uint64_t acc_full;
   __shared__ uint32_t tmem_slot;
 
   const uint32_t base = (smem_u32(dsmem) + 1023u) & ~1023u;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tile = blockIdx.x, m_tile = blockIdx.y;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int m_pair = static_cast<int>(blockIdx.x >> 1), n_tile = static_cast<int>(blockIdx.y);
+  const int m0 = m_pair * (2 * kRowsCta) + static_cast<int>(rank) * kRowsCta;
+  const int64_t w0 = static_cast<int64_t>(n_tile) * kBN + static_cast<int64_t>(rank) * kWRows;
   const int total = p.num_main + p.num_lora;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full_a[s], 1);
-      mbar_init(&full_b[s], kGroupWarps);
+      mbar_init(&xfull[s], 1);
+      mbar_init(&cfull[s], 1);
+      mbar_init(&wfull[s], 2 * kGroupWarps);
       mbar_init(&empty[s], 1);
     }
-    for (int g = 0; g < kGroups; ++g)
-      for (int c = 0; c < kCodeSlots; ++c) {
-        mbar_init(&c_full[g][c], 1);
-        mbar_init(&c_empty[g][c], kGroupWarps);
-      }
-    mbar_init(&acc_bar, 1);
+    mbar_init(&acc_full, 1);
     fence_mbar_init();
     tma_prefetch_desc(&p.tmA);
     tma_prefetch_desc(&p.tmCodes);
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
                  "r"(kTmemCols)
                  : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
+  // Both CTAs' barriers are initialised before either CTA counts bytes or
+  // arrivals on the other's.
+  cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
 
@@ -106,77 +126,77 @@ __global__ void __launch_bounds__(kThreads, 1) fused_fwd_kernel(const __grid_con
       int issued = 0;
       for (int it = 0; it < total; ++it) {
         const int s = it % kStages;
-        if (!mbar_wait_bounded(&empty[s], (static_cast<uint32_t>(it / kStages) & 1u) ^ 1u, p.err, kErrTimeoutEmpty))
-          break;
-        const uint32_t a_s = base + static_cast<uint32_t>(s) * kStageBytes;
+        const uint32_t use = static_cast<uint32_t>(it / kStages);
+        if (!mbar_wait_bounded(&empty[s], (use & 1u) ^ 1u, p.err, kErrTimeoutEmpty)) break;
+        const uint32_t st = base + static_cast<uint32_t>(s) * kStageBytes;
         const bool lora = it >= p.num_main;
         // The adapter operand T comes from the preceding projection kernel.
         if (lora && it == p.num_main && p.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
-        mbar_arrive_expect_tx(&full_a[s], kABytes);
+        const uint32_t xbar = mapa_shared(smem_u32(&xfull[s]), 0);
+        if (leader) mbar_arrive_expect_tx(&xfull[s], 2u * (kABytes + (lora ? kBBytes : 0u)));
+        const int kx = (lora ? it - p.num_main : it) * kBK;
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
-          tma_load_2d(a_s + h * kASub, lora ? &p.tmA2 : &p.tmA, &full_a[s], (lora ? it - p.num_main : it) * kBK,
-                      m_tile * kBM + h * 128);
-        // The step's codes (or, on an adapter step, a bare arrival) go to the
-        // group that takes it, now that the step's weight slot is free.
-        const int g = it % kGroups, gi = it / kGroups, cs = gi % kCodeSlots;
-        if (!mbar_wait_bounded(&c_empty[g][cs], (static_cast<uint32_t>(gi / kCodeSlots) & 1u) ^ 1u, p.err,
-                               kErrTimeoutEmpty))
-          break;
-        if (!lora) {
-          mbar_arrive_expect_tx(&c_full[g][cs], kCBytes);
-          tma_load_2d(base + kCOff + static_cast<uint32_t>(g * kCodeSlots + cs) * kCBytes, &p.tmCodes, &c_full[g][cs],
-                      it * 32, n_tile * kBN);
+        for (int h = 0; h < 2; ++h) {
+          // A 128-row half entirely past m loads rows 0..127 instead: its
+          // accumulator rows are never stored, and every box stays in range.
+          const int y = (m0 + h * 128 < p.m) ? m0 + h * 128 : 0;
+          tma_load_2d_pair(st + h * kASub, lora ? &p.tmA2 : &p.tmA, xbar, kx, y);
+        }
+        const int wy = (w0 < p.n) ? static_cast<int>(w0) : 0;
+        if (lora) {
+          tma_load_2d_pair(st + kBOff, &p.tmB2, xbar, kx, wy);
+          mbar_arrive(&cfull[s]);
         } else {
-          mbar_arrive(&c_full[g][cs]);
+          mbar_arrive_expect_tx(&cfull[s], kCBytes);
+          tma_load_2d(st + kCOff, &p.tmCodes, &cfull[s], it * 32, wy);
         }
         ++issued;
       }
-      // Let the last copies land before the CTA may exit.
-      for (int it = issued - kStages < 0 ? 0 : issued - kStages; it < issued; ++it)
-        mbar_wait_bounded(&full_a[it % kStages], static_cast<uint32_t>(it / kStages) & 1u, p.err, kErrTimeoutDrain);
-      for (int it = issued - kGroups * kCodeSlots < 0 ? 0 : issued - kGroups * kCodeSlots; it < issued; ++it) {
-        const int g = it % kGroups, gi = it / kGroups;
-        mbar_wait_bounded(&c_full[g][gi % kCodeSlots], static_cast<uint32_t>(gi / kCodeSlots) & 1u, p.err,
-                          kErrTimeoutDrain);
+      // Let this CTA's last copies land before it may exit (the leader's
+      // xfull also counts the peer's X boxes).
+      for (int it = issued - kStages < 0 ? 0 : issued - kStages; it < issued; ++it) {
+        const uint32_t ph = static_cast<uint32_t>(it / kStages) & 1u;
+        if (leader) mbar_wait_bounded(&xfull[it % kStages], ph, p.err, kErrTimeoutDrain);
+        mbar_wait_bounded(&cfull[it % kStages], ph, p.err, kErrTimeoutDrain);
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
       bool ok = true;
       for (int it = 0; it < total && ok; ++it) {
         const int s = it % kStages;
         const uint32_t ph = static_cast<uint32_t>(it / kStages) & 1u;
-        ok = mbar_wait_bounded(&full_a[s], ph, p.err, kErrTimeoutFullA) &&
-             mbar_wait_bounded(&full_b[s], ph, p.err, kErrTimeoutFullB);
+        ok = mbar_wait_cluster_bounded(&xfull[s], ph, p.err, kErrTimeoutFullA) &&
+             mbar_wait_cluster_bounded(&wfull[s], ph, p.err, kErrTimeoutFullB);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t a_s = base + static_cast<uint32_t>(s) * kStageBytes;
-        const uint32_t b_s = a_s + kABytes;
+        const uint32_t st = base + static_cast<uint32_t>(s) * kStageBytes;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = smem_desc(a_s + h * kASub + kk * 32u, 16u, 1024u);
-            const uint64_t bd = smem_desc(b_s + kk * 32u, 16u, 1024u);
-            umma_f16(tmem + static_cast<uint32_t>(h * kBN), ad, bd, kIdesc, (it > 0 || kk > 0) ? 1u : 0u);
+            const uint64_t ad = smem_desc(st + h * kASub + kk * 32u, 16u, 1024u);
+            const uint64_t bd = smem_desc(st + kBOff + kk * 32u, 16u, 1024u);
+            umma_f16_pair(tmem + static_cast<uint32_t>(h * kBN), ad, bd, kIdesc, (it > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        umma_commit(&empty[s]);
+        umma_commit_pair_both(&empty[s]);
       }
-      if (ok) umma_commit(&acc_bar);
+      if (ok) umma_commit_pair_both(&acc_full);
     }
   } else {
     // ------------------------------------------------------------ dequant
-    const int grp = (warp - 2) / kGroupWarps;
-    const int dt = (threadIdx.x - 64) & (32 * kGroupWarps - 1);   // weight row of the tile
+    const int dq = warp - 2;
+    const int grp = dq / kGroupWarps;                     // == the stage this group fills
+    const int dt = (dq % kGroupWarps) * 32 + lane;        // weight row of this CTA's half tile
     const int64_t kblocks = p.k / 64;
-    const int64_t gn = static_cast<int64_t>(n_tile) * kBN + dt;
+    const int64_t gn = w0 + dt;
     const bool row_ok = gn < p.n;
     const uint32_t row_off = static_cast<uint32_t>(dt) * 128u;
     const uint32_t sw = static_cast<uint32_t>(dt & 7);
     const uint32_t first_half = ((lane >> 2) & 1u) ? 16u : 0u;
+    const uint32_t wbar = mapa_shared(smem_u32(&wfull[grp]), 0);
     // Absmax code and group scale of this group's next k-step, fetched one
     // step of the group ahead; t = fp32(S / 255) recomputed only when the
     // group index changes (a thread walks one weight row).
@@ -185,18 +205,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_fwd_kernel(const __grid_con
     int64_t g_cur = -1;
     float t_cur = 0.f;
     for (int it = grp; it < total; it += kGroups) {
-      const int gi = it / kGroups, cs = gi % kCodeSlots;
-      if (!mbar_wait_bounded(&c_full[grp][cs], static_cast<uint32_t>(gi / kCodeSlots) & 1u, p.err, kErrTimeoutFullA))
-        break;
-      const uint32_t b_s = base + static_cast<uint32_t>(it % kStages) * kStageBytes + kABytes;
-      const uint32_t rowaddr = b_s + row_off;
+      const uint32_t use = static_cast<uint32_t>(it / kStages);
+      if (!mbar_wait_bounded(&cfull[grp], use & 1u, p.err, kErrTimeoutFullA)) break;
+      const uint32_t st = base + static_cast<uint32_t>(grp) * kStageBytes;
       if (it < p.num_main) {
-        const uint32_t c_s = base + kCOff + static_cast<uint32_t>(grp * kCodeSlots + cs) * kCBytes;
-        const uint4 f = lds128(c_s + static_cast<uint32_t>(dt) * 32u + first_half);
-        const uint4 g2 = lds128(c_s + static_cast<uint32_t>(dt) * 32u + (16u - first_half));
-        // The codes are in registers: release the code slot.
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&c_empty[grp][cs]);
+        const uint32_t c_s = st + kCOff + static_cast<uint32_t>(dt) * 32u;
+        const uint4 f = lds128(c_s + first_half);
+        const uint4 g2 = lds128(c_s + (16u - first_half));
         const uint32_t qv = q_nx;
         const float S = S_nx;
         const int64_t blk = gn * kblocks + it;
@@ -218,40 +233,29 @@ __global__ void __launch_bounds__(kThreads, 1) fused_fwd_kernel(const __grid_con
         }
         const uint4 lo = first_half ? g2 : f, hi = first_half ? f : g2;
         const uint32_t words[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+        const uint32_t rowaddr = st + kBOff + row_off;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t o[4];
           decode8(words[c], tb, o);
           sts128(rowaddr + ((static_cast<uint32_t>(c) ^ sw) << 4), o);
         }
-      } else {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&c_empty[grp][cs]);
-        // Adapter k-step: row gn of B (r columns), columns [64 l, 64 l + 64).
-        // B is an input of the preceding kernel, not its output: no wait.
-        const int l = it - p.num_main;
-        const uint16_t *src = p.B2 + gn * p.r + static_cast<int64_t>(l) * kBK;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (row_ok && l * kBK + 8 * c < p.r) v = __ldg(reinterpret_cast<const uint4 *>(src) + c);
-          const uint32_t o[4] = {v.x, v.y, v.z, v.w};
-          sts128(rowaddr + ((static_cast<uint32_t>(c) ^ sw) << 4), o);
-        }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
+      // Adapter k-steps: the B rows came by TMA; the arrival keeps the
+      // barrier's phases in step.
       __syncwarp();
-      if (lane == 0) mbar_arrive(&full_b[it % kStages]);
+      if (lane == 0) mbar_arrive_cluster(wbar);
     }
 
     // ------------------------------------------------------------ epilogue
-    if (mbar_wait_bounded(&acc_bar, 0u, p.err, kErrTimeoutAcc, 20000000000ull)) {
+    if (mbar_wait_bounded(&acc_full, 0u, p.err, kErrTimeoutAcc, 20000000000ull)) {
       tc_fence_after();
-      const int ew = warp - 2;
-      const int quad = warp & 3;                      // TMEM lanes this warp may read
-      const int h = ew >> 3;
-      const int c_begin = ((ew >> 2) & 1) * (kBN / 2);
-      const int64_t grow = static_cast<int64_t>(m_tile) * kBM + h * 128 + quad * 32 + lane;
+      const int quad = warp & 3;                          // TMEM lanes this warp may read
+      const int q4 = dq >> 2;                             // column quarter of the 512 columns
+      const int h = q4 >> 1;
+      const int c_begin = (q4 & 1) * (kBN / 2);
+      const int64_t grow = static_cast<int64_t>(m0) + h * 128 + quad * 32 + lane;
       const bool out_ok = grow < p.m;
       for (int c0 = c_begin; c0 < c_begin + kBN / 2; c0 += 32) {
         uint32_t v[32];
@@ -277,11 +281,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_fwd_kernel(const __grid_con
     }
   }
 
+  // Neither CTA leaves (or frees tensor memory) while the other may still
+  // count on its barriers or its tensor memory.
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
   }
 }
 
@@ -292,9 +299,11 @@ cudaError_t fused_fwd_large(const uint16_t *X, int64_t m, const WeightView &w, c
   FwdParams p{};
   const bool lora = T != nullptr && B != nullptr && r > 0;
   if (!encode_bf16_map(&p.tmA, X, m, w.k, 64, 128)) return cudaErrorInvalidValue;
-  if (!encode_codes_map(&p.tmCodes, w.codes, w.n, w.k / 2, 32, kBN, false)) return cudaErrorInvalidValue;
-  if (lora && !encode_bf16_map(&p.tmA2, T, m, r, 64, 128)) return cudaErrorInvalidValue;
-  p.B2 = B;
+  if (!encode_codes_map(&p.tmCodes, w.codes, w.n, w.k / 2, 32, kWRows, false)) return cudaErrorInvalidValue;
+  if (lora) {
+    if (!encode_bf16_map(&p.tmA2, T, m, r, 64, 128)) return cudaErrorInvalidValue;
+    if (!encode_bf16_map(&p.tmB2, B, w.n, r, 64, kWRows)) return cudaErrorInvalidValue;
+  }
   p.absmax_q = w.absmax_q;
   p.group_scale = w.group_scale;
   p.out = Y;
@@ -308,25 +317,25 @@ cudaError_t fused_fwd_large(const uint16_t *X, int64_t m, const WeightView &w, c
   p.pdl = (lora && pdl) ? 1 : 0;
   p.tab = *w.tab;
 
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static std::atomic<bool> configured[kMaxDevicesPerProcess] = {};
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(fused_fwd_kernel), static_cast<int>(kSmemBytes),
+                                configured);
   if (e != cudaSuccess) return e;
-  static bool configured[64] = {};
-  if (dev < 0 || dev >= 64 || !configured[dev]) {
-    e = cudaFuncSetAttribute(fused_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) configured[dev] = true;
-  }
+  const int64_t pairs_m = (m + 2 * kRowsCta - 1) / (2 * kRowsCta);
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>((w.n + kBN - 1) / kBN), static_cast<unsigned>((m + kBM - 1) / kBM), 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs_m), static_cast<unsigned>((w.n + kBN - 1) / kBN), 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = p.pdl ? 1 : 0;
+  cfg.numAttrs = p.pdl ? 2 : 1;
   e = cudaLaunchKernelEx(&cfg, fused_fwd_kernel, p);
   if (e == cudaSuccess) count_launches(1);
   return e;
