@@ -117,7 +117,7 @@ def profile_traffic(src_digest: str):
 def kernel_source_digest() -> str:
     import hashlib
     h = hashlib.sha256()
-    for name in ("fused_fwd.cu", "tcgen05.cuh", "common.cuh"):
+    for name in ("fused_pair.cu", "tcgen05.cuh", "common.cuh"):
         with open(os.path.join(ROOT, "bit_nf4_quantized_qlora_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -717,7 +717,7 @@ def run_ours(args):
     traffic = profile_traffic(kernel_source_digest())
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
-                "kernel": "fused_fwd_kernel: NF4 dequant + tcgen05 GEMM (forward, 4096x11008x4096, LoRA r=64)",
+                "kernel": "fused_pair_kernel<false>: NF4 dequant + tcgen05 pair GEMM (forward, 4096x11008x4096, LoRA r=64)",
                 "flops_per_launch": f_launch, "launch_us": round(t_launch * 1e6, 2),
                 "peak_kind": f"{peak_kind} burst bf16 (cuBLAS 8192^3, best of 10)",
                 "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),

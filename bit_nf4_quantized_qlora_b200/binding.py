@@ -98,6 +98,16 @@ _SIGNATURES = {
     "qlora_linear_fwd_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(NF4WeightC),
                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_float,
                                                 ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_lora_dropout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_float,
+                                          ctypes.c_uint64, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_linear_fwd_dropout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(NF4WeightC),
+                                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_float,
+                                                ctypes.c_float, ctypes.c_uint64, ctypes.c_uint64, ctypes.c_void_p,
+                                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "qlora_linear_bwd_dx_dropout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(NF4WeightC),
+                                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_float,
+                                                   ctypes.c_float, ctypes.c_uint64, ctypes.c_uint64, ctypes.c_void_p,
+                                                   ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "qlora_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_selftest_div255": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_uint32, ctypes.c_void_p, ctypes.c_void_p]),
 }
@@ -319,6 +329,56 @@ def qlora_lora_bwd(X: torch.Tensor, dY: torch.Tensor, A: torch.Tensor, B: torch.
            lib().qlora_lora_bwd(X.data_ptr(), dY.data_ptr(), m, n, k, A.data_ptr(), B.data_ptr(), r, float(scale),
                                 dA.data_ptr(), dB.data_ptr(), _ptr(ws), ws_bytes, _stream(stream)))
     return dA, dB
+
+
+def qlora_lora_dropout(X: torch.Tensor, p: float, seed: int, offset: int, out: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+    """Xd = bf16(D . X . fp32(1 / fp32(1 - p))) with the counter-based keep
+    mask of (seed, offset); X bf16 [m x k]."""
+    _need_cuda(X, out)
+    m, k = X.shape
+    if out is None:
+        out = torch.empty_like(X)
+    _check("qlora_lora_dropout", lib().qlora_lora_dropout(X.data_ptr(), m, k, float(p), int(seed), int(offset),
+                                                          out.data_ptr(), _stream(stream)))
+    return out
+
+
+def qlora_linear_fwd_dropout(X: torch.Tensor, w: NF4Weight, A: torch.Tensor, B: torch.Tensor, r: int, scale: float,
+                             p: float, seed: int, offset: int, out: Optional[torch.Tensor] = None,
+                             Xd: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                             stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(Y, Xd): Y = bf16(X . W^T + bf16(s Xd A^T) . B^T) with Xd the dropout of X."""
+    _need_cuda(X, A, B, out, Xd, ws)
+    m = X.shape[0]
+    if out is None:
+        out = torch.empty(m, w.n, dtype=torch.bfloat16, device=X.device)
+    if Xd is None:
+        Xd = torch.empty_like(X)
+    ws, ws_bytes = _workspace(QLORA_OP_FWD, m, w.n, w.k, r, ws, X.device)
+    ws_c = w.c_struct()
+    _check("qlora_linear_fwd_dropout",
+           lib().qlora_linear_fwd_dropout(X.data_ptr(), m, ctypes.byref(ws_c), _ptr(A), _ptr(B), r, float(scale),
+                                          float(p), int(seed), int(offset), Xd.data_ptr(), out.data_ptr(), _ptr(ws),
+                                          ws_bytes, _stream(stream)))
+    return out, Xd
+
+
+def qlora_linear_bwd_dx_dropout(dY: torch.Tensor, w: NF4Weight, A: torch.Tensor, B: torch.Tensor, r: int,
+                                scale: float, p: float, seed: int, offset: int, out: Optional[torch.Tensor] = None,
+                                ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """dX = bf16(bf16(dY . W^) + D . (U . A) . fp32(1 / fp32(1 - p))), U = bf16(s dY B)."""
+    _need_cuda(dY, A, B, out, ws)
+    m = dY.shape[0]
+    if out is None:
+        out = torch.empty(m, w.k, dtype=torch.bfloat16, device=dY.device)
+    ws, ws_bytes = _workspace(QLORA_OP_BWD_DX, m, w.n, w.k, r, ws, dY.device)
+    ws_c = w.c_struct()
+    _check("qlora_linear_bwd_dx_dropout",
+           lib().qlora_linear_bwd_dx_dropout(dY.data_ptr(), m, ctypes.byref(ws_c), _ptr(A), _ptr(B), r, float(scale),
+                                             float(p), int(seed), int(offset), out.data_ptr(), _ptr(ws), ws_bytes,
+                                             _stream(stream)))
+    return out
 
 
 def qlora_linear_fwd_noalloc(X: torch.Tensor, w: NF4Weight, A: Optional[torch.Tensor] = None,

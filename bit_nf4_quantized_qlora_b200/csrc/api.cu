@@ -5,6 +5,7 @@
 #include <atomic>
 #include <climits>
 #include <cstdint>
+#include <cmath>
 #include <cstring>
 
 #include "../../include/qlora.h"
@@ -65,6 +66,20 @@ WeightView view(const qlora_nf4_weight *w) {
 }
 
 constexpr int kMaxDevices = kMaxDevicesPerProcess;
+
+// The dropout constants of probability p: threshold = round_half_even(fp32(p)
+// . 65536) for the 16-bit keep test, keep_scale = fp32(1 / fp32(1 - p)).
+// False unless 0 <= p < 1.
+bool dropout_params(float p, uint64_t seed, uint64_t offset, DropoutParams *d) {
+  if (!(p >= 0.0f && p < 1.0f)) return false;
+  d->seed = seed;
+  d->offset = offset;
+  d->threshold = static_cast<uint32_t>(std::nearbyint(static_cast<double>(p) * 65536.0));
+  const float one = 1.0f;
+  const volatile float q = one - p;   // rounded to fp32 before the division
+  d->keep_scale = one / q;
+  return true;
+}
 
 }  // namespace
 
@@ -136,15 +151,15 @@ int validate_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w, const 
   return QLORA_OK;
 }
 
-int launch_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w, const uint16_t *A, const uint16_t *B,
-               int32_t r, float scale, uint16_t *Y, uint16_t *T, cudaStream_t s) {
+int launch_fwd(const uint16_t *X, const uint16_t *Xa, int64_t m, const qlora_nf4_weight *w, const uint16_t *A,
+               const uint16_t *B, int32_t r, float scale, uint16_t *Y, uint16_t *T, cudaStream_t s) {
   const bool lora = T != nullptr;
   cudaError_t e = cudaSuccess;
   // The main kernel overlaps the adapter projection (programmatic dependent
   // launch) unless the caller is timing the main kernel alone.
   const bool pdl = lora && t_prof_start == nullptr;
   if (m <= kSmallM) {
-    if (lora) e = launch_lora_proj_small(X, m, w->k, A, r, scale, T, s);
+    if (lora) e = launch_lora_proj_small(Xa, m, w->k, A, r, scale, T, s);
     if (e == cudaSuccess) e = prof_mark(t_prof_start, s);
     if (e == cudaSuccess) {
       // Decode sizes take the per-warp streaming kernel; the rest (m > 4,
@@ -156,7 +171,7 @@ int launch_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w, const ui
                                 lora ? r : 0, Y, codebook_tables(w->codebook), s, pdl);
     }
   } else {
-    if (lora) e = tc_proj_kmajor(X, m, w->k, A, r, scale, T, s);
+    if (lora) e = tc_proj_kmajor(Xa, m, w->k, A, r, scale, T, s);
     if (e == cudaSuccess) e = prof_mark(t_prof_start, s);
     if (e == cudaSuccess) e = tc_fwd(X, m, view(w), T, lora ? B : nullptr, lora ? r : 0, Y, s, pdl);
   }
@@ -277,7 +292,7 @@ int qlora_linear_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w, co
   if (ws && !aligned16(ws)) return QLORA_ERR_ALIGN;
   st = check_device();
   if (st != QLORA_OK) return st;
-  return launch_fwd(X, m, w, A, B, r, scale, Y, lora ? static_cast<uint16_t *>(ws) : nullptr,
+  return launch_fwd(X, X, m, w, A, B, r, scale, Y, lora ? static_cast<uint16_t *>(ws) : nullptr,
                     reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -341,6 +356,71 @@ int qlora_lora_bwd(const uint16_t *X, const uint16_t *dY, int64_t m, int64_t n, 
   if (e == cudaSuccess) e = tc_proj_mnmajor(dY, m, n, B, r, scale, U, s);  // U = bf16(s dY B)
   if (e == cudaSuccess) e = tc_tn_skinny(X, m, k, U, r, dA, true, s);      // dA = U^T X
   if (e == cudaSuccess) e = tc_tn_skinny(dY, m, n, T, r, dB, false, s);    // dB = dY^T T
+  return cuda_status(e);
+}
+
+int qlora_lora_dropout(const uint16_t *X, int64_t m, int64_t k, float p, uint64_t seed, uint64_t offset,
+                       uint16_t *Xd, qlora_stream_t stream) {
+  DropoutParams d{};
+  if (!dropout_params(p, seed, offset, &d)) return QLORA_ERR_SHAPE;
+  if (m < 0 || k <= 0 || (k % 64) != 0 || m > (int64_t(1) << 31) || k > (int64_t(1) << 31)) return QLORA_ERR_SHAPE;
+  if (m == 0) return QLORA_OK;
+  if (!X || !Xd) return QLORA_ERR_NULL;
+  if (!aligned16(X) || !aligned16(Xd)) return QLORA_ERR_ALIGN;
+  int st = check_device();
+  if (st != QLORA_OK) return st;
+  return cuda_status(launch_dropout_apply(X, m * k, d, Xd, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int qlora_linear_fwd_dropout(const uint16_t *X, int64_t m, const qlora_nf4_weight *w, const uint16_t *A,
+                             const uint16_t *B, int32_t r, float scale, float p, uint64_t seed, uint64_t offset,
+                             uint16_t *Xd, uint16_t *Y, void *ws, size_t ws_bytes, qlora_stream_t stream) {
+  bool lora = false;
+  int st = validate_fwd(X, m, w, A, B, r, Y, &lora);
+  if (st != QLORA_OK) return st;
+  if (!lora) return A == nullptr || B == nullptr ? QLORA_ERR_NULL : QLORA_ERR_SHAPE;
+  DropoutParams d{};
+  if (!dropout_params(p, seed, offset, &d)) return QLORA_ERR_SHAPE;
+  if (m == 0) return QLORA_OK;
+  if (!Xd) return QLORA_ERR_NULL;
+  if (!aligned16(Xd)) return QLORA_ERR_ALIGN;
+  const size_t need = qlora_workspace_bytes(QLORA_OP_FWD, m, w->n, w->k, r);
+  if (ws == nullptr || ws_bytes < need) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
+  st = check_device();
+  if (st != QLORA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = cuda_status(launch_dropout_apply(X, m * w->k, d, Xd, s));
+  if (st != QLORA_OK) return st;
+  return launch_fwd(X, Xd, m, w, A, B, r, scale, Y, static_cast<uint16_t *>(ws), s);
+}
+
+int qlora_linear_bwd_dx_dropout(const uint16_t *dY, int64_t m, const qlora_nf4_weight *w, const uint16_t *A,
+                                const uint16_t *B, int32_t r, float scale, float p, uint64_t seed, uint64_t offset,
+                                uint16_t *dX, void *ws, size_t ws_bytes, qlora_stream_t stream) {
+  int st = check_weight(w);
+  if (st != QLORA_OK) return st;
+  bool lora = false;
+  st = check_adapter(A, B, r, &lora);
+  if (st != QLORA_OK) return st;
+  if (!lora) return A == nullptr || B == nullptr ? QLORA_ERR_NULL : QLORA_ERR_SHAPE;
+  DropoutParams d{};
+  if (!dropout_params(p, seed, offset, &d)) return QLORA_ERR_SHAPE;
+  if (m < 0 || m > (int64_t(1) << 31)) return QLORA_ERR_SHAPE;
+  if (m == 0) return QLORA_OK;
+  if (!dY || !dX) return QLORA_ERR_NULL;
+  if (!aligned16(dY) || !aligned16(dX)) return QLORA_ERR_ALIGN;
+  const size_t need = qlora_workspace_bytes(QLORA_OP_BWD_DX, m, w->n, w->k, r);
+  if (ws == nullptr || ws_bytes < need) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
+  st = check_device();
+  if (st != QLORA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint16_t *U = static_cast<uint16_t *>(ws);
+  // dX = bf16(dY . W^) first, then the masked adapter term is added to it.
+  cudaError_t e = tc_proj_mnmajor(dY, m, w->n, B, r, scale, U, s);       // U = bf16(s dY B)
+  if (e == cudaSuccess) e = tc_bwd_dx(dY, m, view(w), nullptr, nullptr, 0, dX, s, false);
+  if (e == cudaSuccess) e = tc_dropout_add(U, m, r, A, w->k, d, dX, s);
   return cuda_status(e);
 }
 

@@ -47,9 +47,24 @@ int validate_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w, const 
                  int32_t r, uint16_t *Y, bool *use_adapter);
 
 // Launches a validated forward (m > 0) with T as the rank-r scratch (null:
-// no adapter); returns a qlora status.
-int launch_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w, const uint16_t *A, const uint16_t *B,
-               int32_t r, float scale, uint16_t *Y, uint16_t *T, cudaStream_t s);
+// no adapter); Xa is the adapter's input (X itself, or its dropout); returns
+// a qlora status.
+int launch_fwd(const uint16_t *X, const uint16_t *Xa, int64_t m, const qlora_nf4_weight *w, const uint16_t *A,
+               const uint16_t *B, int32_t r, float scale, uint16_t *Y, uint16_t *T, cudaStream_t s);
+
+// LoRA dropout on the adapter input: keep an element when its 16-bit draw is
+// >= threshold = round(fp32(p) . 65536); a kept element is scaled by
+// keep_scale = fp32(1 / fp32(1 - p)).  The draws come from the counter-based
+// generator of philox.cuh keyed by (seed, offset).
+struct DropoutParams {
+  uint64_t seed, offset;
+  uint32_t threshold;
+  float keep_scale;
+};
+
+// Xd = bf16(D . X . keep_scale), +0 where dropped; numel % 16 == 0.
+cudaError_t launch_dropout_apply(const uint16_t *X, int64_t numel, const DropoutParams &d, uint16_t *Xd,
+                                 cudaStream_t stream);
 
 // TMA tensor maps (2D, row-major).  bf16: 128-byte swizzle.  codes: uint8
 // rows of packed codes, optional 128-byte swizzle.  False if encoding failed.
@@ -102,14 +117,21 @@ struct WeightView {
 cudaError_t tc_fwd(const uint16_t *X, int64_t m, const WeightView &w, const uint16_t *T,
                    const uint16_t *B, int32_t r, uint16_t *Y, cudaStream_t stream, bool pdl);
 
-// The same for m > 128: 256 x 256 tiles, separate rings for the X tile, the
-// packed codes and the dequantized weight tile (fused_fwd.cu).
+// The same for m > 128: 512 x 256 tiles on CTA pairs (fused_pair.cu).
 cudaError_t fused_fwd_large(const uint16_t *X, int64_t m, const WeightView &w, const uint16_t *T,
                             const uint16_t *B, int32_t r, uint16_t *Y, cudaStream_t stream, bool pdl);
+
+// The same for m > 128 on CTA pairs (fused_pair.cu).
+cudaError_t fused_bwd_dx_large(const uint16_t *dY, int64_t m, const WeightView &w, const uint16_t *U,
+                               const uint16_t *A, int32_t r, uint16_t *dX, cudaStream_t stream, bool pdl);
 
 // dX = bf16(dY . W^ + U . A); U may be null.
 cudaError_t tc_bwd_dx(const uint16_t *dY, int64_t m, const WeightView &w, const uint16_t *U,
                       const uint16_t *A, int32_t r, uint16_t *dX, cudaStream_t stream, bool pdl);
+
+// dX = bf16(dX + D . (U . A) . keep_scale) for U [m x r], A [r x k], k % 64 == 0.
+cudaError_t tc_dropout_add(const uint16_t *U, int64_t m, int32_t r, const uint16_t *A, int64_t k,
+                           const DropoutParams &d, uint16_t *dX, cudaStream_t stream);
 
 // Adapter merge W' = W^ + scale * B . A (B [n x r], A [r x k], r % 16 == 0,
 // r <= 256; r == 0 gives W^), written as bf16 and/or fp32 [n x k].

@@ -93,6 +93,6 @@ extern "C" int qlora_linear_fwd_noalloc(const uint16_t *X, int64_t m, const qlor
     const cudaError_t e = qlora::scratch_address(&scratch);
     if (e != cudaSuccess) return qlora::status_from_cuda(e);
   }
-  return qlora::launch_fwd(X, m, w, A, B, r, scale, Y, static_cast<uint16_t *>(scratch),
+  return qlora::launch_fwd(X, X, m, w, A, B, r, scale, Y, static_cast<uint16_t *>(scratch),
                            reinterpret_cast<cudaStream_t>(stream));
 }

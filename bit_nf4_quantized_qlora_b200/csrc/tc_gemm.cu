@@ -39,6 +39,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "philox.cuh"
 #include "tcgen05.cuh"
 
 namespace qlora {
@@ -64,13 +65,20 @@ struct __align__(64) TcParams {
   int pdl;              // launched as a programmatic dependent of the adapter projection
   float alpha;
   Nf4Tables tab;
+  DropoutParams drop;   // masked-add epilogue only
 };
+
+// Epilogues: store bf16(alpha . acc), or (dropout) add the masked product to
+// the bf16 output already there: out = bf16(out + D . acc . keep_scale).
+enum : int { kEpiStore = 0, kEpiDropoutAdd = 1 };
 
 // ---- compile-time configuration -------------------------------------------
 
-template <int BN_, int MSUB_, bool A_MN_, bool B_NF4_, bool B_MN_, bool OUT_T_, bool SPLIT_ = false>
+template <int BN_, int MSUB_, bool A_MN_, bool B_NF4_, bool B_MN_, bool OUT_T_, bool SPLIT_ = false,
+          int EPI_ = kEpiStore>
 struct Cfg {
-  static constexpr bool SPLIT = SPLIT_;   // K split over a cluster, DSMEM reduction
+  static constexpr int EPI = EPI_;
+  static constexpr bool SPLIT = SPLIT_;   // contraction split over a cluster, DSMEM reduction
   static constexpr int BN = BN_;
   static constexpr int MSUB = MSUB_;
   static constexpr bool A_MN = A_MN_;
@@ -98,8 +106,11 @@ struct Cfg {
   static_assert(!(A_MN && MSUB != 1), "MN-major A supports one 128-row tile");
   static_assert(!B_NF4 || BN == 256, "NF4 modes use 256-wide tiles (one block per dequant thread)");
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
-  static_assert(!SPLIT || (!B_NF4 && MSUB == 1 && BN == 64), "split-K is for the skinny products");
-  static_assert(!SPLIT || STAGE_BYTES * STAGES >= 128u * 64u * 4u, "room for the fp32 partial tile");
+  static_assert(!SPLIT || (MSUB == 1 && (B_NF4 ? BN == 256 : BN == 64)),
+                "split-K: the skinny products and the small-M NF4 products");
+  static_assert(!SPLIT || STAGE_BYTES * STAGES >= 128u * static_cast<uint32_t>(BN) * 4u,
+                "room for the fp32 partial tile");
+  static_assert(EPI == kEpiStore || (!SPLIT && !OUT_T && !B_NF4), "masked add: plain row-major output");
 };
 
 template <class C>
@@ -117,18 +128,19 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
   const int lane = threadIdx.x & 31;
   const int n_tile = blockIdx.x;
   const int m_tile = blockIdx.y;
-  // With split-K, CTA z of the cluster runs k-steps [it_begin, it_end).
+  // With split-K, CTA z of the cluster runs k-steps [it_begin, total); the
+  // adapter k-steps, if any, go to the last CTA.
   int it_begin = 0, total = p.num_main + p.num_lora;
   if (C::SPLIT) {
     const int z = static_cast<int>(blockIdx.z), nz = static_cast<int>(gridDim.z);
     it_begin = static_cast<int>((static_cast<int64_t>(p.num_main) * z) / nz);
-    total = static_cast<int>((static_cast<int64_t>(p.num_main) * (z + 1)) / nz);
+    if (z + 1 < nz) total = static_cast<int>((static_cast<int64_t>(p.num_main) * (z + 1)) / nz);
   }
   const int n_iters = total - it_begin;
 
   // A skinny projection lets the kernel that consumes its output launch now;
   // that kernel waits for this grid before it reads the output.
-  if (C::SPLIT) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (C::SPLIT && !C::B_NF4) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full_a[s], 1);
@@ -276,7 +288,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
       // step of the group (DQ_GROUPS k-steps) ahead.  The group constant
       // t = fp32(S / 255) is recomputed only when the group index changes
       // (in the forward a thread walks one weight row, so that is rare).
-      int64_t blk_nx = grp < p.num_main ? block_of(grp) : -1;
+      int64_t blk_nx = it_begin + grp < p.num_main ? block_of(it_begin + grp) : -1;
       uint32_t q_nx = blk_nx >= 0 ? __ldg(p.absmax_q + blk_nx) : 0u;
       float S_nx = blk_nx >= 0 ? __ldg(p.group_scale + (blk_nx >> 8)) : 0.f;
       int64_t g_cur = -1;
@@ -286,9 +298,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
       // group count), so that a group waits on every phase of its stages'
       // barriers and a parity wait cannot be satisfied by an older phase.
       static_assert(C::DQ_GROUPS <= 1 || C::STAGES % C::DQ_GROUPS == 0, "stages per dequant group");
-      for (int it = grp; it < total; it += kStride) {
-        const int s = it % C::STAGES;
-        const uint32_t ph = static_cast<uint32_t>(it / C::STAGES) & 1u;
+      for (int li = grp; li < n_iters; li += kStride) {
+        const int it = it_begin + li;
+        const int s = li % C::STAGES;
+        const uint32_t ph = static_cast<uint32_t>(li / C::STAGES) & 1u;
         if (!mbar_wait_bounded(&full_a[s], ph, p.err, kErrTimeoutFullA)) { ok = false; break; }
         if (it < p.num_main) {
           const int64_t blk = blk_nx;
@@ -377,6 +390,32 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
           continue;
         }
         const int64_t gcol = static_cast<int64_t>(n_tile) * C::BN + c0;
+        if (C::EPI == kEpiDropoutAdd) {
+          // 32 outputs starting at a multiple of 32 of a row whose length is
+          // a multiple of 64: two whole mask blocks, never past the row.
+          if (row_ok && gcol < p.out_cols) {
+            uint16_t *dst = p.out + grow * p.out_ld + gcol;
+            const uint64_t blk = static_cast<uint64_t>(grow * p.out_ld + gcol) >> 4;
+            const uint32_t keep = dropout_keep_bits(blk, p.drop.seed, p.drop.offset, p.drop.threshold) |
+                                  (dropout_keep_bits(blk + 1, p.drop.seed, p.drop.offset, p.drop.threshold) << 16);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint4 old = reinterpret_cast<const uint4 *>(dst)[j];
+              const uint32_t ow[4] = {old.x, old.y, old.z, old.w};
+              uint32_t nw[4];
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                const int e = 8 * j + 2 * t;
+                const float a0 = (keep >> e) & 1u ? __fmul_rn(__uint_as_float(v[e]), p.drop.keep_scale) : 0.f;
+                const float a1 =
+                    (keep >> (e + 1)) & 1u ? __fmul_rn(__uint_as_float(v[e + 1]), p.drop.keep_scale) : 0.f;
+                nw[t] = pack_bf16x2(__fadd_rn(bf16lo_to_f32(ow[t]), a0), __fadd_rn(bf16hi_to_f32(ow[t]), a1));
+              }
+              reinterpret_cast<uint4 *>(dst)[j] = make_uint4(nw[0], nw[1], nw[2], nw[3]);
+            }
+          }
+          continue;
+        }
         if (!C::OUT_T) {
           if (row_ok) {
             uint16_t *dst = p.out + grow * p.out_ld + gcol;
@@ -412,10 +451,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
   __syncthreads();
   if (C::SPLIT) {
     // Reduce the cluster's partial tiles through distributed shared memory:
-    // CTA `rank` finishes rows [rank*128/size, (rank+1)*128/size).
+    // CTA `rank` finishes rows [rank*v/size, (rank+1)*v/size) of the tile's
+    // v rows that exist in the output.
     cluster_sync_all();
     const uint32_t rank = cluster_rank(), size = cluster_size();
-    const int r_lo = static_cast<int>((128u * rank) / size), r_hi = static_cast<int>((128u * (rank + 1)) / size);
+    const int64_t left = static_cast<int64_t>(p.out_rows) - static_cast<int64_t>(m_tile) * C::BM;
+    const uint32_t valid = static_cast<uint32_t>(left < 128 ? (left > 0 ? left : 0) : 128);
+    const int r_lo = static_cast<int>((valid * rank) / size), r_hi = static_cast<int>((valid * (rank + 1)) / size);
     const int rows = r_hi - r_lo;
     for (int i = threadIdx.x; i < rows * C::BN; i += C::NUM_THREADS) {
       const int col = i / rows, row = r_lo + (i % rows);
@@ -477,14 +519,15 @@ cudaError_t launch(const TcParams &p, int grid_n, int grid_m, cudaStream_t strea
   return e;
 }
 
-// Split of the contraction for a skinny product with `tiles` output tiles and
-// `ksteps` k-steps: fill about two CTAs per SM, at least two k-steps per CTA,
-// at most 8 CTAs per cluster.
-int choose_split(int64_t tiles, int ksteps) {
+// Split of the contraction for a product with `tiles` output tiles and
+// `ksteps` k-steps: fill about `per_sm` CTAs per SM (two for the skinny
+// products, which fit two to an SM; one for the input gradient), at least two
+// k-steps per CTA, at most 8 CTAs per cluster.
+int choose_split(int64_t tiles, int ksteps, int per_sm = 2) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int64_t sp = (2LL * sms) / (tiles > 0 ? tiles : 1);
+  int64_t sp = (static_cast<int64_t>(per_sm) * sms) / (tiles > 0 ? tiles : 1);
   if (sp > 8) sp = 8;
   if (sp > ksteps / 2) sp = ksteps / 2;
   return sp < 1 ? 1 : static_cast<int>(sp);
@@ -493,12 +536,14 @@ int choose_split(int64_t tiles, int ksteps) {
 int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
 using CfgFwd1 = Cfg<256, 1, false, true, false, false>;
-using CfgBwd2 = Cfg<256, 2, false, true, true, false>;
+using CfgFwd1S = Cfg<256, 1, false, true, false, false, true>;
 using CfgBwd1 = Cfg<256, 1, false, true, true, false>;
+using CfgBwd1S = Cfg<256, 1, false, true, true, false, true>;
 using CfgProjK = Cfg<64, 1, false, false, false, false, true>;
 using CfgProjMN = Cfg<64, 1, false, false, true, false, true>;
 using CfgTN = Cfg<64, 1, true, false, true, false, true>;
 using CfgTNT = Cfg<64, 1, true, false, true, true, true>;
+using CfgDropAdd = Cfg<256, 1, false, false, true, false, false, kEpiDropoutAdd>;
 
 }  // namespace
 
@@ -530,14 +575,19 @@ cudaError_t tc_fwd(const uint16_t *X, int64_t m, const WeightView &w, const uint
   p.alpha = 1.0f;
   p.tab = *w.tab;
   const int gn = cdiv(w.n, 256), gm = cdiv(m, bm);
-  return launch<CfgFwd1>(p, gn, gm, stream, 1, p.pdl != 0);
+  // Few 256-row weight tiles leave SMs idle: split the contraction over a
+  // cluster (the adapter k-steps go to its last CTA).
+  const int sp = choose_split(int64_t(gn) * gm, p.num_main, 1);
+  return sp > 1 ? launch<CfgFwd1S>(p, gn, gm, stream, sp, p.pdl != 0)
+                : launch<CfgFwd1>(p, gn, gm, stream, 1, p.pdl != 0);
 }
 
 cudaError_t tc_bwd_dx(const uint16_t *dY, int64_t m, const WeightView &w, const uint16_t *U, const uint16_t *A,
                       int32_t r, uint16_t *dX, cudaStream_t stream, bool pdl) {
+  // Above 128 rows: the CTA-pair kernel.
+  if (m > 128) return fused_bwd_dx_large(dY, m, w, U, A, r, dX, stream, pdl);
   TcParams p{};
-  const bool big = m > 128;
-  const uint32_t bm = big ? 256u : 128u;
+  const uint32_t bm = 128u;
   const bool lora = U != nullptr && A != nullptr && r > 0;
   if (!encode_bf16_map(&p.tmA, dY, m, w.n, 64, 128)) return cudaErrorInvalidValue;
   if (!encode_codes_map(&p.tmCodes, w.codes, w.n, w.k / 2, 32, 64, false)) return cudaErrorInvalidValue;
@@ -560,8 +610,11 @@ cudaError_t tc_bwd_dx(const uint16_t *dY, int64_t m, const WeightView &w, const 
   p.alpha = 1.0f;
   p.tab = *w.tab;
   const int gn = cdiv(w.k, 256), gm = cdiv(m, bm);
-  return big ? launch<CfgBwd2>(p, gn, gm, stream, 1, p.pdl != 0)
-             : launch<CfgBwd1>(p, gn, gm, stream, 1, p.pdl != 0);
+  // One 128-row tile per 256 columns leaves most SMs idle at small m: the
+  // contraction over the weight rows is split over a cluster instead.
+  const int sp = choose_split(int64_t(gn) * gm, p.num_main, 1);
+  return sp > 1 ? launch<CfgBwd1S>(p, gn, gm, stream, sp, p.pdl != 0)
+                : launch<CfgBwd1>(p, gn, gm, stream, 1, p.pdl != 0);
 }
 
 cudaError_t tc_proj_kmajor(const uint16_t *L, int64_t m, int64_t kc, const uint16_t *R, int32_t r, float scale,
@@ -614,6 +667,29 @@ cudaError_t tc_tn_skinny(const uint16_t *Lt, int64_t mc, int64_t pdim, const uin
   const int gn = cdiv(r, 64), gm = cdiv(pdim, 128);
   const int sp = choose_split(int64_t(gn) * gm, p.num_main);
   return transposed ? launch<CfgTNT>(p, gn, gm, stream, sp) : launch<CfgTN>(p, gn, gm, stream, sp);
+}
+
+}  // namespace qlora
+
+namespace qlora {
+
+// dX[m x k] = bf16(dX + D . (U . A) . keep_scale): U [m x r] (K-major), A [r x k]
+// (MN-major), the mask regenerated from (seed, offset) over dX's flat index.
+cudaError_t tc_dropout_add(const uint16_t *U, int64_t m, int32_t r, const uint16_t *A, int64_t k,
+                           const DropoutParams &d, uint16_t *dX, cudaStream_t stream) {
+  TcParams p{};
+  if (!encode_bf16_map(&p.tmA, U, m, r, 64, 128)) return cudaErrorInvalidValue;
+  if (!encode_bf16_map(&p.tmB, A, r, k, 64, 64)) return cudaErrorInvalidValue;
+  p.out = dX;
+  p.err = device_error_word();
+  p.out_ld = k;
+  p.out_rows = static_cast<int>(m);
+  p.out_cols = static_cast<int>(k);
+  p.num_main = cdiv(r, 64);
+  p.num_lora = 0;
+  p.alpha = 1.0f;
+  p.drop = d;
+  return launch<CfgDropAdd>(p, cdiv(k, 256), cdiv(m, 128), stream);
 }
 
 }  // namespace qlora

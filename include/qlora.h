@@ -22,7 +22,8 @@
  * Entry points: qlora_quantize_nf4_dq / qlora_quantize_4bit_dq (fp32 W ->
  * codes), qlora_dequant (codes -> bf16 W^), qlora_linear_fwd (and its
  * _noalloc form), qlora_linear_bwd_dx, qlora_lora_bwd (adapter gradients),
- * qlora_merge_adapter (W^ + s B A for export); helpers for workspace sizes,
+ * qlora_merge_adapter (W^ + s B A for export), qlora_lora_dropout and the
+ * _dropout forms of the forward and input gradient; helpers for workspace sizes,
  * codebook levels, errors, versions and launch counts.
  *
  * Conventions for every entry point
@@ -205,6 +206,39 @@ int qlora_lora_bwd(const uint16_t *X, const uint16_t *dY, int64_t m, int64_t n, 
                    const uint16_t *A, const uint16_t *B, int32_t r, float scale,
                    uint16_t *dA, uint16_t *dB, void *ws, size_t ws_bytes,
                    qlora_stream_t stream);
+
+/* LoRA dropout on the adapter input ["QLoRA and Quantized Training", In code:
+ * LoraConfig(r=16, lora_alpha=32, lora_dropout=0.05, ...)].  The pages give
+ * only the probability; the reading taken is inverted dropout on the
+ * adapter's input, as in the LoRA configuration they use:
+ *     Xd = D . X . c,   c = fp32(1 / fp32(1 - p)),   kept: bf16_rne(fp32(x . c)), dropped: +0
+ *     Y  = X . W^T + s . (Xd . A^T) . B^T              (the frozen product keeps X)
+ *     dX = dY . W^ + D . (s . (dY . B) . A) . c
+ *     dA = s . (dY . B)^T . Xd,   dB = s . dY^T . (Xd . A^T)   (qlora_lora_bwd with Xd for X)
+ * The keep mask D is counter-based, so the backward regenerates it from the
+ * forward's (seed, offset): element e of the row-major [m x k] tensor draws
+ * 16-bit lane e % 16 (bits 16 (i % 4) of word i / 4 for lane i) of
+ * Philox4x64-10 (Salmon et al., SC 2011) for counter (e / 16, offset, 0, 0)
+ * under key (seed, 0), and is kept when that value is >= round_half_even(
+ * fp32(p) . 65536).  `offset` separates the masks of different calls (steps,
+ * layers).  0 <= p < 1, else QLORA_ERR_SHAPE; k % 64 == 0.
+ *
+ * qlora_lora_dropout:       Xd [m x k] bf16 from X [m x k] bf16.
+ * qlora_linear_fwd_dropout: writes Xd (keep it for the backward) and Y; an
+ *   adapter is required (A, B non-NULL, r > 0); ws as for qlora_linear_fwd.
+ * qlora_linear_bwd_dx_dropout: dX as above, computed as
+ *   bf16(bf16(dY . W^) + D . (U . A) . c) with U = bf16(s . dY . B); an
+ *   adapter is required; ws as for qlora_linear_bwd_dx.                     */
+int qlora_lora_dropout(const uint16_t *X, int64_t m, int64_t k, float p, uint64_t seed, uint64_t offset,
+                       uint16_t *Xd, qlora_stream_t stream);
+int qlora_linear_fwd_dropout(const uint16_t *X, int64_t m, const qlora_nf4_weight *w,
+                             const uint16_t *A, const uint16_t *B, int32_t r, float scale,
+                             float p, uint64_t seed, uint64_t offset, uint16_t *Xd, uint16_t *Y,
+                             void *ws, size_t ws_bytes, qlora_stream_t stream);
+int qlora_linear_bwd_dx_dropout(const uint16_t *dY, int64_t m, const qlora_nf4_weight *w,
+                                const uint16_t *A, const uint16_t *B, int32_t r, float scale,
+                                float p, uint64_t seed, uint64_t offset, uint16_t *dX,
+                                void *ws, size_t ws_bytes, qlora_stream_t stream);
 
 /* Forward with no caller workspace, for callers that cannot allocate device
  * memory: code whose host owns every device allocation (an engine plugin), a

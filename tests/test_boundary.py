@@ -240,3 +240,36 @@ def test_device_error_bits_match_the_header():
     for name in ("OPERANDS", "WEIGHT_TILE", "FREE_STAGE", "ACCUMULATOR", "DRAIN", "SELFTEST"):
         m = re.search(r"QLORA_DEVERR_%s\s*=\s*1u\s*<<\s*(\d+)" % name, text)
         assert m and getattr(B, "QLORA_DEVERR_" + name) == 1 << int(m.group(1)), name
+
+
+def test_dropout_entry_points_reject_bad_arguments(lib):
+    d = lambda **kw: lib.qlora_lora_dropout(kw.get("X", P), kw.get("m", 16), kw.get("k", 128), kw.get("p", 0.05),
+                                            1, 2, kw.get("Xd", P), None)
+    assert d(p=1.0) == B.QLORA_ERR_SHAPE
+    assert d(p=-0.1) == B.QLORA_ERR_SHAPE
+    assert d(p=float("nan")) == B.QLORA_ERR_SHAPE
+    assert d(k=100) == B.QLORA_ERR_SHAPE
+    assert d(X=None) == B.QLORA_ERR_NULL
+    assert d(Xd=MIS) == B.QLORA_ERR_ALIGN
+    assert d(m=0, X=None, Xd=None) == B.QLORA_OK
+    w = _w()
+    f = lambda **kw: lib.qlora_linear_fwd_dropout(kw.get("X", P), kw.get("m", 16), ctypes.byref(kw.get("w", w)),
+                                                  kw.get("A", P), kw.get("B", P), kw.get("r", 16), 2.0,
+                                                  kw.get("p", 0.05), 1, 2, kw.get("Xd", P), kw.get("Y", P),
+                                                  kw.get("ws", P), kw.get("ws_bytes", 1 << 20), None)
+    assert f(A=None, B=None) == B.QLORA_ERR_NULL                  # dropout needs an adapter
+    assert f(r=0) == B.QLORA_ERR_SHAPE
+    assert f(p=1.5) == B.QLORA_ERR_SHAPE
+    assert f(Xd=None) == B.QLORA_ERR_NULL
+    assert f(Xd=MIS) == B.QLORA_ERR_ALIGN
+    assert f(ws=None) == B.QLORA_ERR_WORKSPACE
+    assert f(w=_w(k=1000)) == B.QLORA_ERR_SHAPE
+    g = lambda **kw: lib.qlora_linear_bwd_dx_dropout(kw.get("dY", P), kw.get("m", 16), ctypes.byref(kw.get("w", w)),
+                                                     kw.get("A", P), kw.get("B", P), kw.get("r", 16), 2.0,
+                                                     kw.get("p", 0.05), 1, 2, kw.get("dX", P), kw.get("ws", P),
+                                                     kw.get("ws_bytes", 1 << 20), None)
+    assert g(B=None) == B.QLORA_ERR_NULL
+    assert g(p=1.0) == B.QLORA_ERR_SHAPE
+    assert g(dX=MIS) == B.QLORA_ERR_ALIGN
+    assert g(ws_bytes=10) == B.QLORA_ERR_WORKSPACE
+    assert g(m=0, dY=None, dX=None) == B.QLORA_OK
