@@ -38,7 +38,7 @@ METRIC = "fused NF4 linear TFLOPS (M=4096) and weight-GB/s (M=1) vs B200 rooflin
 UNIT = "TFLOP/s"
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "fused_fwd_gemm_7b_mlp.txt")
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "fused_pair_fwd_7b_mlp_gate.txt")
 
 
 # ---------------------------------------------------------------------------
@@ -229,7 +229,7 @@ class Projection:
         self.dX = torch.empty(m, k, dtype=torch.bfloat16, device=dev)
         self.dA, self.dB = grad_view_a, grad_view_b
         self.ws_f = torch.empty(B.qlora_workspace_bytes(B.QLORA_OP_FWD, m, n, k, r), dtype=torch.uint8, device=dev)
-        self.ws_b = torch.empty(B.qlora_workspace_bytes(B.QLORA_OP_BWD_DX, m, n, k, r), dtype=torch.uint8, device=dev)
+        self.T = self.ws_f[:m * r * 2].view(torch.bfloat16).view(m, r)
         self.ws_g = torch.empty(B.qlora_workspace_bytes(B.QLORA_OP_LORA_BWD, m, n, k, r), dtype=torch.uint8,
                                 device=dev)
 
@@ -243,8 +243,10 @@ class Projection:
         B.qlora_linear_fwd(self.X, self.w, self.A, self.B, c.r, c.scale, out=self.Y, ws=self.ws_f)
         if prof is not None:
             B.qlora_set_profile_events(None, None)
-        B.qlora_linear_bwd_dx(self.dY, self.w, self.A, self.B, c.r, c.scale, out=self.dX, ws=self.ws_b)
-        B.qlora_lora_bwd(self.X, self.dY, self.A, self.B, c.r, c.scale, dA=self.dA, dB=self.dB, ws=self.ws_g)
+        # Input gradient and adapter gradients in one call; T comes from the
+        # forward's workspace, U is formed once for dX and dA.
+        B.qlora_linear_bwd(self.dY, self.X, self.w, self.A, self.B, c.r, c.scale, T=self.T, dX=self.dX, dA=self.dA,
+                           dB=self.dB, ws=self.ws_g)
 
 
 def _grad_buffer(cases, dev):

@@ -98,6 +98,10 @@ _SIGNATURES = {
     "qlora_linear_fwd_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(NF4WeightC),
                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_float,
                                                 ctypes.c_void_p, ctypes.c_void_p]),
+    "qlora_linear_bwd": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                        ctypes.POINTER(NF4WeightC), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                        ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                        ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "qlora_lora_dropout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_float,
                                           ctypes.c_uint64, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_linear_fwd_dropout": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(NF4WeightC),
@@ -329,6 +333,30 @@ def qlora_lora_bwd(X: torch.Tensor, dY: torch.Tensor, A: torch.Tensor, B: torch.
            lib().qlora_lora_bwd(X.data_ptr(), dY.data_ptr(), m, n, k, A.data_ptr(), B.data_ptr(), r, float(scale),
                                 dA.data_ptr(), dB.data_ptr(), _ptr(ws), ws_bytes, _stream(stream)))
     return dA, dB
+
+
+def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, w: NF4Weight, A: torch.Tensor, B: torch.Tensor, r: int,
+                     scale: float, T: Optional[torch.Tensor] = None, dX: Optional[torch.Tensor] = None,
+                     dA: Optional[torch.Tensor] = None, dB: Optional[torch.Tensor] = None, want_dx: bool = True,
+                     ws: Optional[torch.Tensor] = None, stream=None):
+    """(dX or None, dA, dB) of the layer in one call; T = the forward's
+    bf16(s X A^T) (the first m*r*2 bytes of its workspace) or None."""
+    _need_cuda(dY, X, A, B, T, dX, dA, dB, ws)
+    m, k = X.shape
+    n = dY.shape[1]
+    if dX is None and want_dx:
+        dX = torch.empty(m, k, dtype=torch.bfloat16, device=X.device)
+    if dA is None:
+        dA = torch.empty(r, k, dtype=torch.bfloat16, device=X.device)
+    if dB is None:
+        dB = torch.empty(n, r, dtype=torch.bfloat16, device=X.device)
+    ws, ws_bytes = _workspace(QLORA_OP_LORA_BWD, m, n, k, r, ws, X.device)
+    ws_c = w.c_struct()
+    _check("qlora_linear_bwd",
+           lib().qlora_linear_bwd(dY.data_ptr(), X.data_ptr(), _ptr(T), m, ctypes.byref(ws_c), A.data_ptr(),
+                                  B.data_ptr(), r, float(scale), _ptr(dX), dA.data_ptr(), dB.data_ptr(), _ptr(ws),
+                                  ws_bytes, _stream(stream)))
+    return dX, dA, dB
 
 
 def qlora_lora_dropout(X: torch.Tensor, p: float, seed: int, offset: int, out: Optional[torch.Tensor] = None,

@@ -359,6 +359,45 @@ int qlora_lora_bwd(const uint16_t *X, const uint16_t *dY, int64_t m, int64_t n, 
   return cuda_status(e);
 }
 
+int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint16_t *T, int64_t m, const qlora_nf4_weight *w,
+                     const uint16_t *A, const uint16_t *B, int32_t r, float scale, uint16_t *dX, uint16_t *dA,
+                     uint16_t *dB, void *ws, size_t ws_bytes, qlora_stream_t stream) {
+  int st = check_weight(w);
+  if (st != QLORA_OK) return st;
+  if (!A || !B || !dA || !dB) return QLORA_ERR_NULL;
+  if (r <= 0 || r > 256 || (r % 16) != 0) return QLORA_ERR_SHAPE;
+  if (m < 0 || m > (int64_t(1) << 31)) return QLORA_ERR_SHAPE;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(dA) || !aligned16(dB)) return QLORA_ERR_ALIGN;
+  if ((dX && !aligned16(dX)) || (T && !aligned16(T))) return QLORA_ERR_ALIGN;
+  if (m > 0) {
+    if (!X || !dY) return QLORA_ERR_NULL;
+    if (!aligned16(X) || !aligned16(dY)) return QLORA_ERR_ALIGN;
+    const size_t need = qlora_workspace_bytes(QLORA_OP_LORA_BWD, m, w->n, w->k, r);
+    if (ws == nullptr || ws_bytes < need) return QLORA_ERR_WORKSPACE;
+    if (!aligned16(ws)) return QLORA_ERR_ALIGN;
+  }
+  st = check_device();
+  if (st != QLORA_OK) return st;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t n = w->n, k = w->k;
+  if (m == 0) {
+    cudaError_t e = cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * static_cast<size_t>(k) * 2u, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dB, 0, static_cast<size_t>(n) * static_cast<size_t>(r) * 2u, s);
+    return cuda_status(e);
+  }
+  const size_t mr = round_up(static_cast<size_t>(m) * static_cast<size_t>(r) * 2u);
+  uint16_t *U = static_cast<uint16_t *>(ws);
+  uint16_t *Tw = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(ws) + mr);
+  // U once, for the input gradient and for dA; T from the forward when given.
+  cudaError_t e = tc_proj_mnmajor(dY, m, n, B, r, scale, U, s);                       // U = bf16(s dY B)
+  if (e == cudaSuccess && T == nullptr) e = tc_proj_kmajor(X, m, k, A, r, scale, Tw, s);   // T = bf16(s X A^T)
+  if (e == cudaSuccess && dX) e = tc_bwd_dx(dY, m, view(w), U, A, r, dX, s, false);    // dX = dY W^ + U A
+  if (e == cudaSuccess) e = tc_tn_skinny(X, m, k, U, r, dA, true, s);                  // dA = U^T X
+  if (e == cudaSuccess) e = tc_tn_skinny(dY, m, n, T ? T : Tw, r, dB, false, s);       // dB = dY^T T
+  return cuda_status(e);
+}
+
 int qlora_lora_dropout(const uint16_t *X, int64_t m, int64_t k, float p, uint64_t seed, uint64_t offset,
                        uint16_t *Xd, qlora_stream_t stream) {
   DropoutParams d{};

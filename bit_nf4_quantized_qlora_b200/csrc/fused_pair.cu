@@ -289,11 +289,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_pair_kernel(const __grid_co
         const int64_t blk = blk_nx;
         const uint32_t qv = q_nx;
         const float S = S_nx;
-        if (it + kGroups < p.num_main) {
-          blk_nx = block_of(it + kGroups);
-          q_nx = blk_nx >= 0 ? __ldg(p.absmax_q + blk_nx) : 0u;
-          S_nx = blk_nx >= 0 ? __ldg(p.group_scale + (blk_nx >> 8)) : 0.f;
-        }
         // Codes into registers, code slot released, block table built: all
         // before the weight slot is free.
         Bf16Table tb;
@@ -335,6 +330,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_pair_kernel(const __grid_co
       }
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(wbar);
+      // The next k-step's absmax code and group scale, requested only now so
+      // that the proxy fence above never waits for these loads.
+      if (it + kGroups < p.num_main) {
+        blk_nx = block_of(it + kGroups);
+        q_nx = blk_nx >= 0 ? __ldg(p.absmax_q + blk_nx) : 0u;
+        S_nx = blk_nx >= 0 ? __ldg(p.group_scale + (blk_nx >> 8)) : 0.f;
+      }
     }
 
     // ------------------------------------------------------------ epilogue

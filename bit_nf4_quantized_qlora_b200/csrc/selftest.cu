@@ -63,8 +63,11 @@ extern "C" int qlora_selftest_div255(uint32_t first_bits, uint32_t count, unsign
   return status_from_cuda(cudaGetLastError());
 }
 
-static_assert(qlora::kErrTimeoutFullA == QLORA_DEVERR_OPERANDS && qlora::kErrTimeoutFullB == QLORA_DEVERR_WEIGHT_TILE &&
-                  qlora::kErrTimeoutEmpty == QLORA_DEVERR_FREE_STAGE &&
-                  qlora::kErrTimeoutAcc == QLORA_DEVERR_ACCUMULATOR &&
-                  qlora::kErrTimeoutDrain == QLORA_DEVERR_DRAIN && qlora::kErrTimeoutSelfTest == QLORA_DEVERR_SELFTEST,
+constexpr bool same_bit(unsigned kernel_bit, unsigned header_bit) { return kernel_bit == header_bit; }
+static_assert(same_bit(qlora::kErrTimeoutFullA, QLORA_DEVERR_OPERANDS) &&
+                  same_bit(qlora::kErrTimeoutFullB, QLORA_DEVERR_WEIGHT_TILE) &&
+                  same_bit(qlora::kErrTimeoutEmpty, QLORA_DEVERR_FREE_STAGE) &&
+                  same_bit(qlora::kErrTimeoutAcc, QLORA_DEVERR_ACCUMULATOR) &&
+                  same_bit(qlora::kErrTimeoutDrain, QLORA_DEVERR_DRAIN) &&
+                  same_bit(qlora::kErrTimeoutSelfTest, QLORA_DEVERR_SELFTEST),
               "device error bits of the kernels and of the C header");

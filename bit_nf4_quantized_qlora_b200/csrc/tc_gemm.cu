@@ -92,12 +92,16 @@ struct Cfg {
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + CODE_BYTES;
   static constexpr int STAGES_RAW = static_cast<int>((224u * 1024u) / STAGE_BYTES);
   // Skinny (BN=64) configs keep 4 stages so two CTAs fit on an SM.
-  static constexpr int STAGES = B_NF4 ? (STAGES_RAW > 6 ? 6 : STAGES_RAW) : 4;
+  // The masked-add product has at most four k-steps (K = r <= 256): two
+  // stages, so that two CTAs share an SM.
+  static constexpr int STAGES = B_NF4 ? (STAGES_RAW > 6 ? 6 : STAGES_RAW) : (EPI == kEpiDropoutAdd ? 2 : 4);
   static constexpr uint32_t SMEM_BYTES = STAGE_BYTES * STAGES + 1024u;
   // NF4 modes: groups of 8 dequant warps take k-steps in turn (two groups for
   // the K-major forward tile, one for the MN-major input-gradient tile).
   static constexpr int DQ_GROUPS = B_NF4 ? (B_MN ? 1 : 2) : 0;
-  static constexpr int NUM_EPI_WARPS = B_NF4 ? 8 * DQ_GROUPS : 4;
+  // The masked-add epilogue regenerates the dropout mask (one Philox call per
+  // 16 outputs): sixteen warps share that work.
+  static constexpr int NUM_EPI_WARPS = B_NF4 ? 8 * DQ_GROUPS : (EPI == kEpiDropoutAdd ? 16 : 4);
   static constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
   static constexpr uint32_t TMEM_RAW = static_cast<uint32_t>(BN * MSUB);
   static constexpr uint32_t TMEM_COLS = TMEM_RAW <= 32 ? 32 : TMEM_RAW <= 64 ? 64 : TMEM_RAW <= 128 ? 128 : TMEM_RAW <= 256 ? 256 : 512;

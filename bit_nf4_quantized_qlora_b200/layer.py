@@ -4,9 +4,9 @@ decoder block used to measure it inside a transformer layer.
 The frozen base weight is held only in its NF4 + double-quant form and the
 adapters A [r x k], B [n x r] are bf16 parameters ("QLoRA and Quantized
 Training", The idea; "QLoRA", Follow one QLoRA training step): the forward is
-one ``qlora_linear_fwd``, the backward one ``qlora_linear_bwd_dx`` for the
-input gradient and one ``qlora_lora_bwd`` for the adapter gradients, all in
-libqlora's kernels.  The rest of the decoder block (RMSNorm, causal
+one ``qlora_linear_fwd`` and the backward one ``qlora_linear_bwd`` (input
+gradient and adapter gradients, reusing the forward's rank-r intermediate),
+all in libqlora's kernels.  The rest of the decoder block (RMSNorm, causal
 attention, SiLU gating, residual adds) is plain PyTorch: it is not part of
 the quantized layer, and the pages leave it to the host framework.
 """
@@ -23,17 +23,23 @@ class QLoRALinearFunction(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, X: torch.Tensor, A: torch.Tensor, Bm: torch.Tensor, w: B.NF4Weight, r: int, scale: float):
-        Y = B.qlora_linear_fwd(X, w, A, Bm, r, scale)
-        ctx.save_for_backward(X, A, Bm)
+        m = X.shape[0]
+        ws = torch.empty(max(1, B.qlora_workspace_bytes(B.QLORA_OP_FWD, m, w.n, w.k, r)), dtype=torch.uint8,
+                         device=X.device)
+        Y = B.qlora_linear_fwd(X, w, A, Bm, r, scale, ws=ws)
+        # The forward leaves T = bf16(s X A^T) at the start of its workspace;
+        # the backward takes it instead of recomputing it.
+        T = ws[:m * r * 2].view(torch.bfloat16).view(m, r) if r > 0 and m > 0 else None
+        ctx.save_for_backward(X, A, Bm, T)
         ctx.w, ctx.r, ctx.scale = w, r, scale
         return Y
 
     @staticmethod
     def backward(ctx, dY: torch.Tensor):
-        X, A, Bm = ctx.saved_tensors
+        X, A, Bm, T = ctx.saved_tensors
         dY = dY.contiguous()
-        dX = B.qlora_linear_bwd_dx(dY, ctx.w, A, Bm, ctx.r, ctx.scale) if ctx.needs_input_grad[0] else None
-        dA, dB = B.qlora_lora_bwd(X, dY, A, Bm, ctx.r, ctx.scale)
+        dX, dA, dB = B.qlora_linear_bwd(dY, X, ctx.w, A, Bm, ctx.r, ctx.scale, T=T,
+                                        want_dx=ctx.needs_input_grad[0])
         return dX, dA, dB, None, None, None
 
 

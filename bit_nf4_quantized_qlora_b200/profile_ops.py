@@ -26,7 +26,8 @@ WORKLOADS = {
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=("quantize", "dequant", "fwd", "fwd_nolora", "bwd_dx", "lora_bwd", "merge"), required=True)
+    ap.add_argument("--op", choices=("quantize", "dequant", "fwd", "fwd_nolora", "bwd_dx", "lora_bwd", "merge", "dropout",
+                                     "fwd_dropout", "bwd_dx_dropout"), required=True)
     ap.add_argument("--workload", choices=sorted(WORKLOADS), required=True)
     ap.add_argument("--m", type=int, default=4096)
     ap.add_argument("--iters", type=int, default=3)
@@ -42,15 +43,16 @@ def main(argv=None):
         del W
     r = case.r
     X = A = Bm = dY = Y = None
-    if a.op in ("fwd", "fwd_nolora", "lora_bwd"):
+    if a.op in ("fwd", "fwd_nolora", "lora_bwd", "dropout", "fwd_dropout"):
         X = case.X().to(dev)
-    if a.op in ("bwd_dx", "lora_bwd"):
+    if a.op in ("bwd_dx", "lora_bwd", "bwd_dx_dropout"):
         dY = case.dY().to(dev)
     A, Bm = case.A().to(dev), case.B().to(dev)
     out_w = torch.empty(case.n, case.k, dtype=torch.bfloat16, device=dev) if a.op in ("dequant", "merge") else None
-    if a.op in ("fwd", "fwd_nolora"):
+    if a.op in ("fwd", "fwd_nolora", "fwd_dropout"):
         Y = torch.empty(case.m, case.n, dtype=torch.bfloat16, device=dev)
-    if a.op == "bwd_dx":
+    Xd = torch.empty_like(X) if a.op in ("dropout", "fwd_dropout") else None
+    if a.op in ("bwd_dx", "bwd_dx_dropout"):
         Y = torch.empty(case.m, case.k, dtype=torch.bfloat16, device=dev)
 
     def run():
@@ -66,6 +68,12 @@ def main(argv=None):
             B.qlora_linear_fwd(X, w, None, None, 0, 0.0, out=Y)
         elif a.op == "bwd_dx":
             B.qlora_linear_bwd_dx(dY, w, A, Bm, r, case.scale, out=Y)
+        elif a.op == "dropout":
+            B.qlora_lora_dropout(X, 0.05, 1234, 7, out=Xd)
+        elif a.op == "fwd_dropout":
+            B.qlora_linear_fwd_dropout(X, w, A, Bm, r, case.scale, 0.05, 1234, 7, out=Y, Xd=Xd)
+        elif a.op == "bwd_dx_dropout":
+            B.qlora_linear_bwd_dx_dropout(dY, w, A, Bm, r, case.scale, 0.05, 1234, 7, out=Y)
         else:
             B.qlora_lora_bwd(X, dY, A, Bm, r, case.scale)
 

@@ -22,6 +22,7 @@
  * Entry points: qlora_quantize_nf4_dq / qlora_quantize_4bit_dq (fp32 W ->
  * codes), qlora_dequant (codes -> bf16 W^), qlora_linear_fwd (and its
  * _noalloc form), qlora_linear_bwd_dx, qlora_lora_bwd (adapter gradients),
+ * qlora_linear_bwd (the whole backward, rank-r intermediates formed once),
  * qlora_merge_adapter (W^ + s B A for export), qlora_lora_dropout and the
  * _dropout forms of the forward and input gradient; helpers for workspace sizes,
  * codebook levels, errors, versions and launch counts.
@@ -172,7 +173,9 @@ int qlora_merge_adapter(const qlora_nf4_weight *w, const uint16_t *A, const uint
  *   scale  in   s = alpha / r
  *   Y      out  bf16 [m x n]
  *   ws     scratch, ws_bytes >= qlora_workspace_bytes(QLORA_OP_FWD, m, n, k, r);
- *          contents on entry are ignored.
+ *          contents on entry are ignored; when the call returns (in stream
+ *          order) its first m*r*2 bytes hold T [m x r], which
+ *          qlora_linear_bwd can take instead of recomputing it.
  * Products accumulate in fp32.  m <= 16 runs a weight-streaming kernel; larger
  * m runs the tcgen05 tensor-core kernel with dequantization in its main loop. */
 int qlora_linear_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w,
@@ -206,6 +209,24 @@ int qlora_lora_bwd(const uint16_t *X, const uint16_t *dY, int64_t m, int64_t n, 
                    const uint16_t *A, const uint16_t *B, int32_t r, float scale,
                    uint16_t *dA, uint16_t *dB, void *ws, size_t ws_bytes,
                    qlora_stream_t stream);
+
+/* The whole backward of the layer in one call: dX, dA and dB, with the
+ * rank-r intermediates formed once ["QLoRA", Follow one QLoRA training step,
+ * step 4; "QLoRA and Quantized Training", The idea]:
+ *   U  = bf16(s . dY . B)   computed once, used by dX and by dA
+ *   dX = bf16(dY . W^ + U . A)          (skipped when dX is NULL)
+ *   dA = bf16(U^T . X),  dB = bf16(dY^T . T)
+ *   T  = bf16(s . X . A^T): pass the forward's (qlora_linear_fwd leaves it at
+ *        the start of its workspace, [m x r] row-major), or NULL to compute it
+ *        here.  With dropout, X is the forward's Xd and T its workspace.
+ *   dY, X  in   bf16 [m x n], [m x k];  A, B as in the forward, r > 0
+ *   dX, dA, dB out  (dX may be NULL); ws >= qlora_workspace_bytes(QLORA_OP_LORA_BWD, m, n, k, r)
+ * m == 0 writes zeros to dA and dB.  Same results as qlora_linear_bwd_dx
+ * followed by qlora_lora_bwd, with two fewer rank-r projections.           */
+int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint16_t *T, int64_t m,
+                     const qlora_nf4_weight *w, const uint16_t *A, const uint16_t *B, int32_t r,
+                     float scale, uint16_t *dX, uint16_t *dA, uint16_t *dB, void *ws, size_t ws_bytes,
+                     qlora_stream_t stream);
 
 /* LoRA dropout on the adapter input ["QLoRA and Quantized Training", In code:
  * LoraConfig(r=16, lora_alpha=32, lora_dropout=0.05, ...)].  The pages give

@@ -273,3 +273,20 @@ def test_dropout_entry_points_reject_bad_arguments(lib):
     assert g(dX=MIS) == B.QLORA_ERR_ALIGN
     assert g(ws_bytes=10) == B.QLORA_ERR_WORKSPACE
     assert g(m=0, dY=None, dX=None) == B.QLORA_OK
+
+
+def test_linear_bwd_rejects_bad_arguments(lib):
+    w = _w()
+    f = lambda **kw: lib.qlora_linear_bwd(kw.get("dY", P), kw.get("X", P), kw.get("T", None), kw.get("m", 16),
+                                          ctypes.byref(kw.get("w", w)), kw.get("A", P), kw.get("B", P),
+                                          kw.get("r", 16), 2.0, kw.get("dX", P), kw.get("dA", P), kw.get("dB", P),
+                                          kw.get("ws", P), kw.get("ws_bytes", 1 << 20), None)
+    assert f(A=None) == B.QLORA_ERR_NULL
+    assert f(dB=None) == B.QLORA_ERR_NULL
+    assert f(X=None) == B.QLORA_ERR_NULL
+    assert f(r=0) == B.QLORA_ERR_SHAPE
+    assert f(w=_w(k=1000)) == B.QLORA_ERR_SHAPE
+    assert f(dX=MIS) == B.QLORA_ERR_ALIGN
+    assert f(T=MIS) == B.QLORA_ERR_ALIGN
+    assert f(ws=None) == B.QLORA_ERR_WORKSPACE
+    assert f(ws_bytes=100) == B.QLORA_ERR_WORKSPACE

@@ -320,3 +320,30 @@ def test_attn_proj_7b_decode(m):
 
 def test_no_device_timeouts_recorded():
     assert B.qlora_poll_device_error() == 0
+
+
+@pytest.mark.parametrize("nkmr", [(1024, 1024, 16, 16), (520, 640, 200, 32), (776, 1088, 300, 256), (264, 192, 1, 16)],
+                         ids=lambda c: "n%d_k%d_m%d_r%d" % c)
+@pytest.mark.parametrize("reuse_t", [True, False], ids=["T_from_forward", "T_recomputed"])
+def test_linear_bwd_parity(nkmr, reuse_t):
+    """qlora_linear_bwd (dX, dA, dB in one call, U formed once, T from the
+    forward's workspace or recomputed) against the oracle."""
+    n, k, m, r = nkmr
+    case = _case(n, k, m, r, seed=1500)
+    W, X, A, Bm = _inputs(case)
+    dY = case.dY()
+    w = _gpu_quant(W)
+    Xd, Ad, Bd, dYd = X.to(DEV), A.to(DEV), Bm.to(DEV), dY.to(DEV)
+    ws = torch.empty(B.qlora_workspace_bytes(B.QLORA_OP_FWD, m, n, k, r), dtype=torch.uint8, device=DEV)
+    B.qlora_linear_fwd(Xd, w, Ad, Bd, r, case.scale, ws=ws)
+    T = ws[:m * r * 2].view(torch.bfloat16).view(m, r) if reuse_t else None
+    dX, dA, dB = B.qlora_linear_bwd(dYd, Xd, w, Ad, Bd, r, case.scale, T=T)
+    _, dA2, dB2 = B.qlora_linear_bwd(dYd, Xd, w, Ad, Bd, r, case.scale, T=T, want_dx=False)
+    torch.cuda.synchronize()
+    W_hat = R.dequant_full(W)
+    Xf, Af, Bf, dYf = (R.bf16_to_f64(t) for t in (X, A, Bm, dY))
+    assert R.err(R.bf16_to_f64(dX), R.bwd_dx(dYf, W_hat, Af, Bf, case.scale)) <= TOL
+    rA, rB = R.lora_grads(Xf, dYf, Af, Bf, case.scale)
+    for a, b in ((dA, dB), (dA2, dB2)):
+        assert R.err(R.bf16_to_f64(a), rA) <= TOL
+        assert R.err(R.bf16_to_f64(b), rB) <= TOL
