@@ -42,7 +42,8 @@
 //            block's table as soon as the codes land, waits only for the
 //            slot's previous MMAs (the same empty barrier the activation
 //            producer waits on) before writing, and arrives on the leader's
-//            wfull barrier; then the epilogue.
+//            wfull barrier; then the epilogue (accumulators -> bf16 tile in
+//            the idle activation ring -> four TMA stores).
 // So after the MMAs of a stage complete, the activation copy and the weight
 // expansion of the stage's next k-step run side by side, not one after the
 // other.
@@ -86,6 +87,7 @@ struct __align__(64) PairParams {
   CUtensorMap tmCodes;   // codes [n x k/2] bytes; box {32, 128} (forward), {32, 64} (input gradient)
   CUtensorMap tmA2;      // T or U [m x r] bf16, box {64, 128}, 128B swizzle
   CUtensorMap tmB2;      // adapter B [n x r] box {64, 128} (forward); A [r x k] box {64, 64} (input gradient)
+  CUtensorMap tmOut;     // Y [m x n] or dX [m x k] bf16, box {64, 256}, 128B swizzle (TMA stores)
   const uint8_t *absmax_q;
   const float *group_scale;
   uint16_t *out;         // Y [m x n] or dX [m x k]
@@ -340,36 +342,46 @@ __global__ void __launch_bounds__(kThreads, 1) fused_pair_kernel(const __grid_co
     }
 
     // ------------------------------------------------------------ epilogue
-    if (mbar_wait_bounded(&acc_full, 0u, p.err, kErrTimeoutAcc, 20000000000ull)) {
+    // The accumulators go out through shared memory: every operand copy and
+    // MMA of the tile is done once acc_full completes, so the activation
+    // ring (128 KB) holds the CTA's bf16 output tile [256 rows x 256 columns]
+    // as four 64-column slabs of 128-byte rows, 128-byte swizzled (the TMA
+    // box layout; a quarter-warp's 16-byte stores hit eight distinct bank
+    // groups).  Four TMA stores then write whole lines of Y (or dX).
+    const bool acc_ok = mbar_wait_bounded(&acc_full, 0u, p.err, kErrTimeoutAcc, 20000000000ull);
+    if (acc_ok) {
       tc_fence_after();
       const int quad = warp & 3;                          // TMEM lanes this warp may read
       const int q4 = dq >> 2;                             // column quarter of the 512 columns
       const int h = q4 >> 1;
       const int c_begin = (q4 & 1) * (kBN / 2);
-      const int64_t grow = static_cast<int64_t>(m0) + h * 128 + quad * 32 + lane;
-      const bool out_ok = grow < p.m;
+      const uint32_t row = static_cast<uint32_t>(h * 128 + quad * 32 + lane);   // row of the CTA's tile
+      const uint32_t rsw = row & 7u;
       for (int cc = c_begin; cc < c_begin + kBN / 2; cc += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(h * kBN + cc), v);
-        const int64_t gcol = static_cast<int64_t>(n_tile) * kBN + cc;
-        if (!out_ok) continue;
-        uint16_t *dst = p.out + grow * p.out_cols + gcol;
-        if (gcol + 32 <= p.out_cols) {
+        const uint32_t slab_row = base + static_cast<uint32_t>(cc >> 6) * 32768u + row * 128u;
+        const uint32_t c16 = static_cast<uint32_t>((cc & 63) >> 3);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
-            w.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
-            w.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
-            w.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
-            reinterpret_cast<uint4 *>(dst)[j] = w;
-          }
-        } else {
-          for (int j = 0; j < 32; ++j)
-            if (gcol + j < p.out_cols)
-              dst[j] = static_cast<uint16_t>(pack_bf16x2(__uint_as_float(v[j]), 0.f) & 0xFFFFu);
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t w[4] = {pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1])),
+                                 pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                                 pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                                 pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]))};
+          sts128(slab_row + (((c16 + static_cast<uint32_t>(j)) ^ rsw) << 4), w);
         }
       }
+      fence_proxy_async_smem();
+    }
+    // All 16 epilogue warps (512 threads) take part, even after a timeout.
+    named_barrier_sync(1, 32 * kGroups * kGroupWarps);
+    if (dq == 0 && lane == 0 && acc_ok && m0 < p.m) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t col = static_cast<int64_t>(n_tile) * kBN + 64 * j;
+        if (col < p.out_cols) tma_store_2d(&p.tmOut, base + static_cast<uint32_t>(j) * 32768u, static_cast<int>(col), m0);
+      }
+      tma_store_drain();
     }
   }
 
@@ -438,6 +450,7 @@ cudaError_t fused_fwd_large(const uint16_t *X, int64_t m, const WeightView &w, c
     if (!encode_bf16_map(&p.tmA2, T, m, r, 64, 128)) return cudaErrorInvalidValue;
     if (!encode_bf16_map(&p.tmB2, B, w.n, r, 64, kHalfN)) return cudaErrorInvalidValue;
   }
+  if (!encode_bf16_map(&p.tmOut, Y, m, w.n, 64, 256)) return cudaErrorInvalidValue;
   p.out_cols = w.n;
   p.num_main = static_cast<int>(w.k / kBK);
   return launch_pair<false>(p, m, w.n, stream);
@@ -453,6 +466,7 @@ cudaError_t fused_bwd_dx_large(const uint16_t *dY, int64_t m, const WeightView &
     if (!encode_bf16_map(&p.tmA2, U, m, r, 64, 128)) return cudaErrorInvalidValue;
     if (!encode_bf16_map(&p.tmB2, A, r, w.k, 64, 64)) return cudaErrorInvalidValue;
   }
+  if (!encode_bf16_map(&p.tmOut, dX, m, w.k, 64, 256)) return cudaErrorInvalidValue;
   p.out_cols = w.k;
   p.num_main = static_cast<int>((w.n + kBK - 1) / kBK);
   return launch_pair<true>(p, m, w.k, stream);
