@@ -390,9 +390,16 @@ int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint16_t *T, i
   uint16_t *U = static_cast<uint16_t *>(ws);
   uint16_t *Tw = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(ws) + mr);
   // U once, for the input gradient and for dA; T from the forward when given.
-  cudaError_t e = tc_proj_mnmajor(dY, m, n, B, r, scale, U, s);                       // U = bf16(s dY B)
-  if (e == cudaSuccess && T == nullptr) e = tc_proj_kmajor(X, m, k, A, r, scale, Tw, s);   // T = bf16(s X A^T)
-  if (e == cudaSuccess && dX) e = tc_bwd_dx(dY, m, view(w), U, A, r, dX, s, false);    // dX = dY W^ + U A
+  cudaError_t e = cudaSuccess;
+  if (T == nullptr) e = tc_proj_kmajor(X, m, k, A, r, scale, Tw, s);                   // T = bf16(s X A^T)
+  if (e == cudaSuccess) e = tc_proj_mnmajor(dY, m, n, B, r, scale, U, s);              // U = bf16(s dY B)
+  // The input-gradient kernel needs U only for its adapter k-steps: it is
+  // launched as a programmatic dependent of the U projection, which directly
+  // precedes it (unless the caller times the main kernel alone).
+  const bool pdl = t_prof_start == nullptr;
+  if (e == cudaSuccess) e = prof_mark(t_prof_start, s);
+  if (e == cudaSuccess && dX) e = tc_bwd_dx(dY, m, view(w), U, A, r, dX, s, pdl);      // dX = dY W^ + U A
+  if (e == cudaSuccess) e = prof_mark(t_prof_stop, s);
   if (e == cudaSuccess) e = tc_tn_skinny(X, m, k, U, r, dA, true, s);                  // dA = U^T X
   if (e == cudaSuccess) e = tc_tn_skinny(dY, m, n, T ? T : Tw, r, dB, false, s);       // dB = dY^T T
   return cuda_status(e);
