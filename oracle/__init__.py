@@ -26,6 +26,7 @@ Modules:
 * ``codebooks`` -- the FP4 and INT4 baselines beside NF4.
 * ``merge``   -- folding the adapter into the dequantized base (export).
 * ``dropout`` -- LoRA dropout on the adapter input (Philox4x64-10 mask).
+* ``dq_fp8``  -- the mean-subtracted 8-bit-float (E4M3) double quantization.
 
 Every function is pinned by a ``-m "not gpu"`` test in ``tests/test_oracle.py``
 against invariants, closed forms, brute force or a library routine; none is
