@@ -24,12 +24,19 @@ QLORA_ERR_WORKSPACE = -4
 QLORA_ERR_CUDA = -5
 QLORA_ERR_DEVICE = -6
 QLORA_ERR_CODEBOOK = -7
+QLORA_ERR_FORMAT = -8
 
 # 4-bit codebooks (the weight's `codebook`): NF4 and the FP4 / INT4 baselines.
 QLORA_CODEBOOK_NF4 = 0
 QLORA_CODEBOOK_FP4 = 1
 QLORA_CODEBOOK_INT4 = 2
 CODEBOOKS = {"nf4": QLORA_CODEBOOK_NF4, "fp4": QLORA_CODEBOOK_FP4, "int4": QLORA_CODEBOOK_INT4}
+
+# Storage formats of the double-quantized absmax (the weight's `dq_format`):
+# unsigned linear 8-bit codes, or E4M3 offsets from the tensor mean.
+QLORA_DQ_LINEAR8 = 0
+QLORA_DQ_FP8_MEAN = 1
+DQ_FORMATS = {"linear8": QLORA_DQ_LINEAR8, "fp8_mean": QLORA_DQ_FP8_MEAN}
 
 # Bits of the device error word (qlora_poll_device_error).
 QLORA_DEVERR_OPERANDS = 1 << 0
@@ -60,7 +67,8 @@ class QLoRAError(RuntimeError):
 class NF4WeightC(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("absmax_q", ctypes.c_void_p),
                 ("group_scale", ctypes.c_void_p), ("n", ctypes.c_int64), ("k", ctypes.c_int64),
-                ("block", ctypes.c_int32), ("group", ctypes.c_int32), ("codebook", ctypes.c_int32)]
+                ("block", ctypes.c_int32), ("group", ctypes.c_int32), ("codebook", ctypes.c_int32),
+                ("dq_format", ctypes.c_int32)]
 
 
 _LIB = None
@@ -71,6 +79,10 @@ _SIGNATURES = {
     "qlora_quantize_4bit_dq": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
                                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                               ctypes.c_void_p]),
+    "qlora_quantize_4bit_dq_format": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                                     ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
+                                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                     ctypes.c_void_p]),
     "qlora_codebook_levels": (ctypes.c_int, [ctypes.c_int32, ctypes.POINTER(ctypes.c_float)]),
     "qlora_dequant": (ctypes.c_int, [ctypes.POINTER(NF4WeightC), ctypes.c_void_p, ctypes.c_void_p]),
     "qlora_merge_adapter": (ctypes.c_int, [ctypes.POINTER(NF4WeightC), ctypes.c_void_p, ctypes.c_void_p,
@@ -161,14 +173,15 @@ class NF4Weight:
     the device) plus its shape [n x k]."""
     codes: torch.Tensor          # uint8 [n*k/2]
     absmax_q: torch.Tensor       # uint8 [n*k/64]
-    group_scale: torch.Tensor    # float32 [ceil(n*k/64/256)]
+    group_scale: torch.Tensor    # float32 [ceil(n*k/64/256)] (+ the mean, QLORA_DQ_FP8_MEAN)
     n: int
     k: int
     codebook: int = QLORA_CODEBOOK_NF4
+    dq_format: int = QLORA_DQ_LINEAR8
 
     def c_struct(self) -> NF4WeightC:
         return NF4WeightC(self.codes.data_ptr(), self.absmax_q.data_ptr(), self.group_scale.data_ptr(),
-                          self.n, self.k, BLOCK, GROUP, self.codebook)
+                          self.n, self.k, BLOCK, GROUP, self.codebook, self.dq_format)
 
     @property
     def nbytes(self) -> int:
@@ -220,23 +233,30 @@ def qlora_quantize_nf4_dq(W: torch.Tensor, absmax_fp32: Optional[torch.Tensor] =
 
 
 def qlora_quantize_4bit_dq(W: torch.Tensor, codebook: int, absmax_fp32: Optional[torch.Tensor] = None,
-                           out: Optional[NF4Weight] = None, stream=None) -> NF4Weight:
-    """fp32 W [n x k] on the device -> NF4Weight in `codebook` (QLORA_CODEBOOK_*)."""
+                           out: Optional[NF4Weight] = None, stream=None,
+                           dq_format: int = QLORA_DQ_LINEAR8) -> NF4Weight:
+    """fp32 W [n x k] on the device -> NF4Weight in `codebook` (QLORA_CODEBOOK_*)
+    with its absmax stored in `dq_format` (QLORA_DQ_*)."""
     _need_cuda(W, absmax_fp32)
     if W.dtype != torch.float32 or W.dim() != 2:
         raise ValueError("W must be a 2-D float32 tensor")
     n, k = W.shape
     numel = n * k
+    n_scales = max(n_groups(numel), 1) + (1 if dq_format == QLORA_DQ_FP8_MEAN else 0)
     if out is None:
         dev = W.device
         out = NF4Weight(torch.empty(numel // 2, dtype=torch.uint8, device=dev),
                         torch.empty(numel // BLOCK, dtype=torch.uint8, device=dev),
-                        torch.empty(max(n_groups(numel), 1), dtype=torch.float32, device=dev), n, k, codebook)
+                        torch.empty(n_scales, dtype=torch.float32, device=dev), n, k, codebook, dq_format)
     else:
+        if out.group_scale.numel() < n_scales:
+            raise ValueError(f"out.group_scale holds {out.group_scale.numel()} entries, {n_scales} needed")
         out.codebook = codebook
-    _check("qlora_quantize_4bit_dq",
-           lib().qlora_quantize_4bit_dq(W.data_ptr(), n, k, codebook, out.codes.data_ptr(), out.absmax_q.data_ptr(),
-                                        out.group_scale.data_ptr(), _ptr(absmax_fp32), _stream(stream)))
+        out.dq_format = dq_format
+    _check("qlora_quantize_4bit_dq_format",
+           lib().qlora_quantize_4bit_dq_format(W.data_ptr(), n, k, codebook, dq_format, out.codes.data_ptr(),
+                                               out.absmax_q.data_ptr(), out.group_scale.data_ptr(),
+                                               _ptr(absmax_fp32), _stream(stream)))
     return out
 
 

@@ -45,6 +45,7 @@ int check_weight(const qlora_nf4_weight *w, bool linear = true) {
   if (linear && (w->n % 8) != 0) return QLORA_ERR_SHAPE;
   if (w->block != 64 || w->group != 256) return QLORA_ERR_SHAPE;
   if (w->codebook < 0 || w->codebook >= kCodebookCount) return QLORA_ERR_CODEBOOK;
+  if (w->dq_format < 0 || w->dq_format >= kDqFormatCount) return QLORA_ERR_FORMAT;
   if (w->n > (int64_t(1) << 31) || w->k > (int64_t(1) << 31)) return QLORA_ERR_SHAPE;
   if (!aligned16(w->codes) || !aligned16(w->absmax_q) || !aligned16(w->group_scale)) return QLORA_ERR_ALIGN;
   return QLORA_OK;
@@ -62,7 +63,8 @@ int check_adapter(const uint16_t *A, const uint16_t *B, int32_t r, bool *use) {
 }
 
 WeightView view(const qlora_nf4_weight *w) {
-  return WeightView{w->codes, w->absmax_q, w->group_scale, w->n, w->k, &codebook_tables(w->codebook)};
+  return WeightView{w->codes, w->absmax_q, w->group_scale, w->n, w->k, &codebook_tables(w->codebook),
+                    mean_ptr(w->group_scale, w->n * w->k / 64, w->dq_format)};
 }
 
 constexpr int kMaxDevices = kMaxDevicesPerProcess;
@@ -165,10 +167,10 @@ int launch_fwd(const uint16_t *X, const uint16_t *Xa, int64_t m, const qlora_nf4
       // Decode sizes take the per-warp streaming kernel; the rest (m > 4,
       // or K beyond one cluster's warps) the CTA-ring kernel.
       e = gemv_stream_supported(m, w->n, w->k)
-              ? launch_gemv_stream(X, m, w->codes, w->absmax_q, w->group_scale, w->n, w->k, T,
+              ? launch_gemv_stream(X, m, w->codes, w->absmax_q, w->group_scale, view(w).mu, w->n, w->k, T,
                                    lora ? B : nullptr, lora ? r : 0, Y, codebook_tables(w->codebook), s, pdl)
-              : launch_gemv_fwd(X, m, w->codes, w->absmax_q, w->group_scale, w->n, w->k, T, lora ? B : nullptr,
-                                lora ? r : 0, Y, codebook_tables(w->codebook), s, pdl);
+              : launch_gemv_fwd(X, m, w->codes, w->absmax_q, w->group_scale, view(w).mu, w->n, w->k, T,
+                                lora ? B : nullptr, lora ? r : 0, Y, codebook_tables(w->codebook), s, pdl);
     }
   } else {
     if (lora) e = tc_proj_kmajor(Xa, m, w->k, A, r, scale, T, s);
@@ -208,6 +210,7 @@ const char *qlora_status_string(int status) {
     case QLORA_ERR_CUDA: return "QLORA_ERR_CUDA: a CUDA call failed";
     case QLORA_ERR_DEVICE: return "QLORA_ERR_DEVICE: the current device is not sm_100";
     case QLORA_ERR_CODEBOOK: return "QLORA_ERR_CODEBOOK: unknown codebook";
+    case QLORA_ERR_FORMAT: return "QLORA_ERR_FORMAT: unknown absmax storage format";
     default: return "unknown qlora status";
   }
 }
@@ -242,8 +245,16 @@ int qlora_quantize_nf4_dq(const float *W, int64_t n, int64_t k, uint8_t *codes, 
 
 int qlora_quantize_4bit_dq(const float *W, int64_t n, int64_t k, int32_t codebook, uint8_t *codes,
                            uint8_t *absmax_q, float *group_scale, float *absmax_fp32, qlora_stream_t stream) {
+  return qlora_quantize_4bit_dq_format(W, n, k, codebook, QLORA_DQ_LINEAR8, codes, absmax_q, group_scale,
+                                       absmax_fp32, stream);
+}
+
+int qlora_quantize_4bit_dq_format(const float *W, int64_t n, int64_t k, int32_t codebook, int32_t dq_format,
+                                  uint8_t *codes, uint8_t *absmax_q, float *group_scale, float *absmax_fp32,
+                                  qlora_stream_t stream) {
   if (!W || !codes || !absmax_q || !group_scale) return QLORA_ERR_NULL;
   if (codebook < 0 || codebook >= kCodebookCount) return QLORA_ERR_CODEBOOK;
+  if (dq_format < 0 || dq_format >= kDqFormatCount) return QLORA_ERR_FORMAT;
   if (n <= 0 || k <= 0 || (k % 64) != 0) return QLORA_ERR_SHAPE;
   if (n > (int64_t(1) << 40) / k) return QLORA_ERR_SHAPE;
   if (!aligned16(W) || !aligned16(codes) || !aligned16(absmax_q) || !aligned16(group_scale) ||
@@ -252,7 +263,7 @@ int qlora_quantize_4bit_dq(const float *W, int64_t n, int64_t k, int32_t codeboo
   int st = check_device();
   if (st != QLORA_OK) return st;
   return cuda_status(launch_quantize(W, n * k, codes, absmax_q, group_scale, absmax_fp32, codebook_tables(codebook),
-                                     reinterpret_cast<cudaStream_t>(stream)));
+                                     dq_format, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int qlora_merge_adapter(const qlora_nf4_weight *w, const uint16_t *A, const uint16_t *B, int32_t r, float scale,
@@ -278,7 +289,8 @@ int qlora_dequant(const qlora_nf4_weight *w, uint16_t *W_bf16, qlora_stream_t st
   st = check_device();
   if (st != QLORA_OK) return st;
   return cuda_status(launch_dequant(w->codes, w->absmax_q, w->group_scale, w->n * w->k, W_bf16,
-                                    codebook_tables(w->codebook), reinterpret_cast<cudaStream_t>(stream)));
+                                    codebook_tables(w->codebook), w->dq_format,
+                                    reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int qlora_linear_fwd(const uint16_t *X, int64_t m, const qlora_nf4_weight *w, const uint16_t *A,

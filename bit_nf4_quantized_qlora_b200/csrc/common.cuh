@@ -57,6 +57,30 @@ __device__ __forceinline__ float absmax_dequant(uint32_t q, float S) {
   return __fmul_rn(static_cast<float>(q), __fdiv_rn(S, 255.0f));
 }
 
+// The fp32 value of an E4M3 bit pattern (1 sign, 4 exponent bits with bias
+// 7, 3 mantissa bits; exponent field 0 holds m/8 * 2^-6), built from its bits.
+__device__ __forceinline__ float e4m3_to_f32(uint32_t q) {
+  const uint32_t e = (q >> 3) & 15u, m = q & 7u;
+  const float mag = e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : static_cast<float>(m) * 0x1p-9f;
+  return (q & 0x80u) ? -mag : mag;
+}
+
+// The two storage formats of the block absmax (fp8 == false: linear 8-bit;
+// true: E4M3 offsets from the tensor mean mu):
+//   linear 8-bit:  t = fp32(S_g / 255),  c' = fp32(q * t)
+//   E4M3 + mean:   t = S'_g (stored),    c' = fp32(fp32(E4M3(q) * t) + mu)
+// Kernels carry the format as a pointer to mu, null for linear 8-bit.
+__device__ __forceinline__ float group_constant(float stored, bool fp8) {
+  return fp8 ? stored : __fdiv_rn(stored, 255.0f);
+}
+__device__ __forceinline__ float code_value(uint32_t q, bool fp8) {
+  return fp8 ? e4m3_to_f32(q) : static_cast<float>(q);
+}
+__device__ __forceinline__ float block_constant(uint32_t q, float t, bool fp8, float mu) {
+  return fp8 ? __fadd_rn(__fmul_rn(e4m3_to_f32(q), t), mu) : __fmul_rn(static_cast<float>(q), t);
+}
+__device__ __forceinline__ float load_mu(const float *mu) { return mu ? __ldg(mu) : 0.f; }
+
 __device__ __forceinline__ void make_table(const Nf4Tables &tab, float cprime, Bf16Table &t) {
   uint32_t p[8];
 #pragma unroll

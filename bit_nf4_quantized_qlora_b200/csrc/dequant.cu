@@ -21,7 +21,9 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t *__rest
                                                            const float *__restrict__ group_scale,
                                                            int64_t n_half_blocks,
                                                            uint16_t *__restrict__ out,
-                                                           const Nf4Tables tab) {
+                                                           const Nf4Tables tab, const float *mu_ptr) {
+  const bool fp8 = mu_ptr != nullptr;
+  const float mu = load_mu(mu_ptr);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t h = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; h < n_half_blocks;
        h += stride) {
@@ -30,7 +32,7 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t *__rest
     const uint32_t q = absmax_q[blk];
     const float S = __ldg(group_scale + (blk >> 8));
     Bf16Table t;
-    make_table(tab, absmax_dequant(q, S), t);
+    make_table(tab, block_constant(q, group_constant(S, fp8), fp8, mu), t);
     uint32_t o[16];
     decode8(cw.x, t, o + 0);
     decode8(cw.y, t, o + 4);
@@ -47,7 +49,8 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t *__rest
 }  // namespace
 
 cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *absmax_q, const float *group_scale,
-                           int64_t numel, uint16_t *out, const Nf4Tables &tab, cudaStream_t stream) {
+                           int64_t numel, uint16_t *out, const Nf4Tables &tab, int dq_format,
+                           cudaStream_t stream) {
   const int64_t nh = numel / 32;
   if (nh == 0) return cudaSuccess;
   int dev = 0, sms = 148;
@@ -56,7 +59,8 @@ cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *absmax_q, const 
   const int64_t want = (nh + kThreads - 1) / kThreads;
   const int64_t cap = static_cast<int64_t>(sms) * 8;
   const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
-  dequant_kernel<<<grid, kThreads, 0, stream>>>(codes, absmax_q, group_scale, nh, out, tab);
+  dequant_kernel<<<grid, kThreads, 0, stream>>>(codes, absmax_q, group_scale, nh, out, tab,
+                                                mean_ptr(group_scale, numel / 64, dq_format));
   count_launches(1);
   return cudaGetLastError();
 }

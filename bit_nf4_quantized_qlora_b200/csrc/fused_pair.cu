@@ -90,6 +90,7 @@ struct __align__(64) PairParams {
   CUtensorMap tmOut;     // Y [m x n] or dX [m x k] bf16, box {64, 256}, 128B swizzle (TMA stores)
   const uint8_t *absmax_q;
   const float *group_scale;
+  const float *mu;                 // E4M3 + mean absmax format: the tensor mean; else null
   uint16_t *out;         // Y [m x n] or dX [m x k]
   unsigned *err;
   int64_t n, k;          // weight shape
@@ -275,8 +276,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_pair_kernel(const __grid_co
       return (gn < p.n && kb < kblocks) ? gn * kblocks + kb : -1;
     };
     // Absmax code and group scale of this group's next k-step, fetched one
-    // step of the group ahead; t = fp32(S / 255) recomputed only when the
-    // group index changes.
+    // step of the group ahead; the group constant t (fp32(S / 255) for
+    // linear codes) recomputed only when the group index changes.
+    const bool fp8 = p.mu != nullptr;
+    const float mu = load_mu(p.mu);
     int64_t blk_nx = grp < p.num_main ? block_of(grp) : -1;
     uint32_t q_nx = blk_nx >= 0 ? __ldg(p.absmax_q + blk_nx) : 0u;
     float S_nx = blk_nx >= 0 ? __ldg(p.group_scale + (blk_nx >> 8)) : 0.f;
@@ -308,9 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_pair_kernel(const __grid_co
           const int64_t gidx = blk >> 8;
           if (gidx != g_cur) {
             g_cur = gidx;
-            t_cur = __fdiv_rn(S, 255.0f);
+            t_cur = group_constant(S, fp8);
           }
-          make_table(p.tab, __fmul_rn(static_cast<float>(qv), t_cur), tb);
+          make_table(p.tab, block_constant(qv, t_cur, fp8, mu), tb);
         } else {
 #pragma unroll
           for (int j = 0; j < 4; ++j) tb.lo[j] = tb.hi[j] = 0u;
@@ -426,6 +429,7 @@ PairParams common_params(const WeightView &w, int64_t m, int32_t r, bool lora, b
   PairParams p{};
   p.absmax_q = w.absmax_q;
   p.group_scale = w.group_scale;
+  p.mu = w.mu;
   p.out = out;
   p.err = device_error_word();
   p.n = w.n;

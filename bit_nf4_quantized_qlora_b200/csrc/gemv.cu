@@ -44,6 +44,7 @@ struct __align__(64) GemvParams {
   const uint16_t *X;
   const uint8_t *absmax_q;
   const float *group_scale;
+  const float *mu;              // E4M3 + mean absmax format: the tensor mean; else null
   const uint16_t *T;
   const uint16_t *B;
   uint16_t *Y;
@@ -170,8 +171,10 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
       off1[b] = static_cast<uint32_t>(lr1) * 128u + chunk + 8u * (q & 1);
     }
 
-    // t = fp32(S / 255) of each row's current group and the block where the
-    // next group starts.
+    // t (the group constant, fp32(S / 255) for linear 8-bit codes) of each
+    // row's current group and the block where the next group starts.
+    const bool fp8 = p.mu != nullptr;
+    const float mu = load_mu(p.mu);
     float t0 = 0.f, t1 = 0.f;
     int next0 = kb_lo, next1 = kb_lo;
 
@@ -197,17 +200,28 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
       const bool full = kb_st + kStageBlocks <= kblocks;
       // Absmax codes and X of this stage, issued before the wait.
       float qf0[kStageBlocks], qf1[kStageBlocks];
+      bool qv[kStageBlocks];
       if (full && qwords) {
         const uint32_t w0 = __ldg(reinterpret_cast<const uint32_t *>(q0p + st * kStageBlocks));
         const uint32_t w1 = __ldg(reinterpret_cast<const uint32_t *>(q1p + st * kStageBlocks));
-        qf0[0] = byte_to_f32<0>(w0); qf0[1] = byte_to_f32<1>(w0); qf0[2] = byte_to_f32<2>(w0); qf0[3] = byte_to_f32<3>(w0);
-        qf1[0] = byte_to_f32<0>(w1); qf1[1] = byte_to_f32<1>(w1); qf1[2] = byte_to_f32<2>(w1); qf1[3] = byte_to_f32<3>(w1);
+        if (fp8) {
+#pragma unroll
+          for (int b = 0; b < kStageBlocks; ++b) {
+            qf0[b] = e4m3_to_f32((w0 >> (8 * b)) & 0xFFu);
+            qf1[b] = e4m3_to_f32((w1 >> (8 * b)) & 0xFFu);
+          }
+        } else {
+          qf0[0] = byte_to_f32<0>(w0); qf0[1] = byte_to_f32<1>(w0); qf0[2] = byte_to_f32<2>(w0); qf0[3] = byte_to_f32<3>(w0);
+          qf1[0] = byte_to_f32<0>(w1); qf1[1] = byte_to_f32<1>(w1); qf1[2] = byte_to_f32<2>(w1); qf1[3] = byte_to_f32<3>(w1);
+        }
+#pragma unroll
+        for (int b = 0; b < kStageBlocks; ++b) qv[b] = true;
       } else {
 #pragma unroll
         for (int b = 0; b < kStageBlocks; ++b) {
-          const bool v = kb_st + b < kblocks;
-          qf0[b] = v ? static_cast<float>(__ldg(q0p + st * kStageBlocks + b)) : 0.f;
-          qf1[b] = v ? static_cast<float>(__ldg(q1p + st * kStageBlocks + b)) : 0.f;
+          qv[b] = kb_st + b < kblocks;
+          qf0[b] = qv[b] ? code_value(__ldg(q0p + st * kStageBlocks + b), fp8) : 0.f;
+          qf1[b] = qv[b] ? code_value(__ldg(q1p + st * kStageBlocks + b), fp8) : 0.f;
         }
       }
       uint4 xa[kStageBlocks][TOK_TILES], xb[kStageBlocks][TOK_TILES];
@@ -226,11 +240,11 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
       // Group constants: with 4-aligned blocks a group boundary falls on a
       // stage start; otherwise the slow path below takes it block by block.
       if (kb_st >= next0) {
-        t0 = __fdiv_rn(__ldg(p.group_scale + ((b0 + kb_st) >> 8)), 255.0f);
+        t0 = group_constant(__ldg(p.group_scale + ((b0 + kb_st) >> 8)), fp8);
         next0 = kb_st + 256 - static_cast<int>((b0 + kb_st) & 255);
       }
       if (kb_st >= next1) {
-        t1 = __fdiv_rn(__ldg(p.group_scale + ((b1 + kb_st) >> 8)), 255.0f);
+        t1 = group_constant(__ldg(p.group_scale + ((b1 + kb_st) >> 8)), fp8);
         next1 = kb_st + 256 - static_cast<int>((b1 + kb_st) & 255);
       }
       ok = mbar_wait_bounded(&full_bar[s], ph, p.err, kErrTimeoutFullA);
@@ -246,17 +260,17 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
         if (!fast) {
           const int kb = kb_st + b;
           if (kb == next0 && kb < kblocks) {
-            t0 = __fdiv_rn(__ldg(p.group_scale + ((b0 + kb) >> 8)), 255.0f);
+            t0 = group_constant(__ldg(p.group_scale + ((b0 + kb) >> 8)), fp8);
             next0 += 256;
           }
           if (kb == next1 && kb < kblocks) {
-            t1 = __fdiv_rn(__ldg(p.group_scale + ((b1 + kb) >> 8)), 255.0f);
+            t1 = group_constant(__ldg(p.group_scale + ((b1 + kb) >> 8)), fp8);
             next1 += 256;
           }
         }
-        // Blocks past K have q = 0 and add nothing.
-        const float s0 = __fmul_rn(qf0[b], t0);
-        const float s1 = __fmul_rn(qf1[b], t1);
+        // c' of the block (zero past K, where the block adds nothing).
+        const float s0 = qv[b] ? __fadd_rn(__fmul_rn(qf0[b], t0), mu) : 0.f;
+        const float s1 = qv[b] ? __fadd_rn(__fmul_rn(qf1[b], t1), mu) : 0.f;
 #pragma unroll
         for (int t = 0; t < TOK_TILES; ++t) {
           acc[t][0] = fmaf(s0, bacc[t][0], acc[t][0]);
@@ -379,7 +393,7 @@ cudaError_t launch_lora_proj_small(const uint16_t *X, int64_t m, int64_t k, cons
 }
 
 cudaError_t launch_gemv_fwd(const uint16_t *X, int64_t m, const uint8_t *codes, const uint8_t *absmax_q,
-                            const float *group_scale, int64_t n, int64_t k, const uint16_t *T,
+                            const float *group_scale, const float *mu, int64_t n, int64_t k, const uint16_t *T,
                             const uint16_t *B, int32_t r, uint16_t *Y, const Nf4Tables &tab,
                             cudaStream_t stream, bool pdl) {
   if (m <= 0) return cudaSuccess;
@@ -388,6 +402,7 @@ cudaError_t launch_gemv_fwd(const uint16_t *X, int64_t m, const uint8_t *codes, 
   p.X = X;
   p.absmax_q = absmax_q;
   p.group_scale = group_scale;
+  p.mu = mu;
   p.T = T;
   p.B = B;
   p.Y = Y;

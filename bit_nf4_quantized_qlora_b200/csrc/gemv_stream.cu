@@ -75,7 +75,8 @@ struct __align__(64) StreamParams {
   CUtensorMap tmCodes;           // codes [n x k/2] bytes, box {128, tile rows}, 128B swizzle
   CUtensorMap tmQ;               // absmax codes [n x k/64] bytes, box {16, tile rows} (MODE 2)
   const uint8_t *absmax_q;       // [n x k/64]
-  const float *group_scale;      // [ceil(n k / 16384)]
+  const float *group_scale;      // [ceil(n k / 16384)] (+ the tensor mean, E4M3 + mean format)
+  const float *mu;               // E4M3 + mean format: the tensor mean; else null
   const uint16_t *X;             // [m x k] bf16
   const uint16_t *T;             // [m x r] bf16 (adapter intermediate) or null
   const uint16_t *B;             // [n x r] bf16
@@ -166,7 +167,8 @@ __device__ __forceinline__ bool slot_pass(const F &f, uint32_t ph, std::integer_
   return f(ph, std::integral_constant<int, S>{}...);
 }
 
-template <int MODE>
+// FP8: the absmax codes are E4M3 offsets from the tensor mean (p.mu).
+template <int MODE, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_constant__ StreamParams p) {
   extern __shared__ __align__(1024) uint8_t dsmem[];
   const uint8_t *lut = dsmem;
@@ -238,7 +240,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
     for (int j = 0; j < 4; ++j) xf[i][j] = v ? __ldg(xp + j) : make_uint4(0u, 0u, 0u, 0u);
   }
 
-  // fp32(S / 255) of every group the CTA's rows touch.  Rows of the last
+  // The group constant t (fp32(S / 255) for linear codes) of every group
+  // the CTA's rows touch.  Rows of the last
   // tile past n (codes and absmax codes read as zero) index the table too;
   // their entries repeat the last group.  Row * k/64 fits in 32 bits
   // (checked on the host).  The first group scale of each thread is loaded
@@ -251,9 +254,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
                             : 0.f;
   build_pair_lut(dsmem, p.tab, threadIdx.x, kThreads);
   for (int i = threadIdx.x; i < nt * kTileRows * kMaxM; i += kThreads) red[i] = 0.f;
-  if (static_cast<int>(threadIdx.x) < ngroups) ttab[threadIdx.x] = div255_rn(s_first);
+  const auto gconst = [](float stored) { return FP8 ? stored : div255_rn(stored); };
+  if (static_cast<int>(threadIdx.x) < ngroups) ttab[threadIdx.x] = gconst(s_first);
   for (int i = threadIdx.x + kThreads; i < ngroups; i += kThreads)
-    ttab[i] = div255_rn(__ldg(p.group_scale + min(gbase + i, glast)));
+    ttab[i] = gconst(__ldg(p.group_scale + min(gbase + i, glast)));
+  const float mu = FP8 ? __ldg(p.mu) : 0.f;
   __syncthreads();
 
   if (active) {
@@ -330,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
 #pragma unroll
         for (int j = 0; j < 2 * kSub; ++j) qw[j] = lds32(qring_w + S * kQSlot + qoff + 128u * j);
       }
-      float acc[2 * kSub];
+      float acc[2 * kSub], dsum[2 * kSub];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         float d[kSub][4];
@@ -347,23 +352,33 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
 #pragma unroll
         for (int j = 0; j < 2 * kSub; ++j) {
           const float da = d[j >> 1][2 * (j & 1)], db = d[j >> 1][2 * (j & 1) + 1];
-          const float qa = i == 0 ? byte_to_f32<0>(qw[j]) : byte_to_f32<2>(qw[j]);
-          const float qb = i == 0 ? byte_to_f32<1>(qw[j]) : byte_to_f32<3>(qw[j]);
+          float qa, qb;
+          if (FP8) {
+            qa = e4m3_to_f32((qw[j] >> (16 * i)) & 0xFFu);
+            qb = e4m3_to_f32((qw[j] >> (16 * i + 8)) & 0xFFu);
+          } else {
+            qa = i == 0 ? byte_to_f32<0>(qw[j]) : byte_to_f32<2>(qw[j]);
+            qb = i == 0 ? byte_to_f32<1>(qw[j]) : byte_to_f32<3>(qw[j]);
+          }
           if (MODE != 0) {
-            // One group per chunk: fp32(S/255) is common to the four blocks
-            // and is applied once per row below.
+            // One group per chunk: t is common to the four blocks and is
+            // applied once per row below, the mean term (E4M3 + mean) as
+            // mu times the sum of the raw block products.
             acc[j] = i == 0 ? qa * da : fmaf(qa, da, acc[j]);
             acc[j] = fmaf(qb, db, acc[j]);
+            if (FP8) dsum[j] = i == 0 ? da + db : dsum[j] + da + db;
           } else {
             const float ta = 2 * i < split[j] ? tlo[j] : thi[j], tb = 2 * i + 1 < split[j] ? tlo[j] : thi[j];
-            acc[j] = i == 0 ? __fmul_rn(qa, ta) * da : fmaf(__fmul_rn(qa, ta), da, acc[j]);
-            acc[j] = fmaf(__fmul_rn(qb, tb), db, acc[j]);
+            const float ca = FP8 ? __fadd_rn(__fmul_rn(qa, ta), mu) : __fmul_rn(qa, ta);
+            const float cb = FP8 ? __fadd_rn(__fmul_rn(qb, tb), mu) : __fmul_rn(qb, tb);
+            acc[j] = i == 0 ? ca * da : fmaf(ca, da, acc[j]);
+            acc[j] = fmaf(cb, db, acc[j]);
           }
         }
       }
       if (MODE != 0) {
 #pragma unroll
-        for (int j = 0; j < 2 * kSub; ++j) acc[j] *= tlo[j];
+        for (int j = 0; j < 2 * kSub; ++j) acc[j] = FP8 ? fmaf(dsum[j], mu, acc[j] * tlo[j]) : acc[j] * tlo[j];
       }
       // The slot's bytes are consumed: refill it with the unit kStages ahead.
       __syncwarp();
@@ -434,20 +449,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
   cluster_sync_all();
 }
 
-template <int MODE>
+template <int MODE, bool FP8>
 cudaError_t configure(int dev) {
-  static bool done[64] = {};
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (done[dev]) return cudaSuccess;
-  const cudaError_t e = cudaFuncSetAttribute(gemv_stream_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(kSmemBytes));
-  if (e == cudaSuccess) done[dev] = true;
-  return e;
+  static std::atomic<bool> done[kMaxDevicesPerProcess] = {};
+  if (dev < 0 || dev >= kMaxDevicesPerProcess) return cudaErrorInvalidDevice;
+  return set_smem_once(reinterpret_cast<const void *>(gemv_stream_kernel<MODE, FP8>), static_cast<int>(kSmemBytes),
+                       &done[dev]);
 }
 
-template <int MODE>
+template <int MODE, bool FP8>
 cudaError_t launch_mode(const StreamParams &p, int dev, int sms, int cs, cudaStream_t stream, bool pdl) {
-  cudaError_t e = configure<MODE>(dev);
+  cudaError_t e = configure<MODE, FP8>(dev);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(cs), 1, 1);
@@ -466,20 +478,22 @@ cudaError_t launch_mode(const StreamParams &p, int dev, int sms, int cs, cudaStr
   // One CTA per SM: as many clusters as can be resident at once (the GPC
   // layout may hold fewer than sms / cs), each with a contiguous run of at
   // most kMaxTiles tiles.
-  static int resident[64][kMaxCluster + 1] = {};
-  int &res = resident[dev][cs];
+  static std::atomic<int> resident[kMaxDevicesPerProcess][2][kMaxCluster + 1] = {};
+  if (dev >= kMaxDevicesPerProcess) return cudaErrorInvalidDevice;
+  int res = resident[dev][FP8 ? 1 : 0][cs].load(std::memory_order_relaxed);
   if (res == 0) {
     int v = 0;
-    e = cudaOccupancyMaxActiveClusters(&v, gemv_stream_kernel<MODE>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&v, gemv_stream_kernel<MODE, FP8>, &cfg);
     if (e != cudaSuccess) return e;
     res = v > 0 ? v : (sms / cs > 0 ? sms / cs : 1);
+    resident[dev][FP8 ? 1 : 0][cs].store(res, std::memory_order_relaxed);
   }
   int ncl = res < p.ntiles ? res : p.ntiles;
   const int min_ncl = (p.ntiles + kMaxTiles - 1) / kMaxTiles;
   if (ncl < min_ncl) ncl = min_ncl;
   cfg.gridDim = dim3(static_cast<unsigned>(cs), static_cast<unsigned>(ncl), 1);
   cfg.numAttrs = (p.r > 0 && pdl) ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, gemv_stream_kernel<MODE>, p);
+  return cudaLaunchKernelEx(&cfg, gemv_stream_kernel<MODE, FP8>, p);
 }
 
 }  // namespace
@@ -490,7 +504,7 @@ bool gemv_stream_supported(int64_t m, int64_t n, int64_t k) {
 }
 
 cudaError_t launch_gemv_stream(const uint16_t *X, int64_t m, const uint8_t *codes, const uint8_t *absmax_q,
-                               const float *group_scale, int64_t n, int64_t k, const uint16_t *T,
+                               const float *group_scale, const float *mu, int64_t n, int64_t k, const uint16_t *T,
                                const uint16_t *B, int32_t r, uint16_t *Y, const Nf4Tables &tab,
                                cudaStream_t stream, bool pdl) {
   if (m <= 0) return cudaSuccess;
@@ -502,6 +516,7 @@ cudaError_t launch_gemv_stream(const uint16_t *X, int64_t m, const uint8_t *code
   if (mode == 2 && !encode_codes_map(&p.tmQ, absmax_q, n, kblocks, 16, kTileRows, false)) return cudaErrorInvalidValue;
   p.absmax_q = absmax_q;
   p.group_scale = group_scale;
+  p.mu = mu;
   p.X = X;
   p.T = T;
   p.B = B;
@@ -520,9 +535,11 @@ cudaError_t launch_gemv_stream(const uint16_t *X, int64_t m, const uint8_t *code
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const cudaError_t e = mode == 2   ? launch_mode<2>(p, dev, sms, cs, stream, pdl)
-                        : mode == 1 ? launch_mode<1>(p, dev, sms, cs, stream, pdl)
-                                    : launch_mode<0>(p, dev, sms, cs, stream, pdl);
+  const bool fp8 = mu != nullptr;
+  const cudaError_t e =
+      mode == 2   ? (fp8 ? launch_mode<2, true>(p, dev, sms, cs, stream, pdl) : launch_mode<2, false>(p, dev, sms, cs, stream, pdl))
+      : mode == 1 ? (fp8 ? launch_mode<1, true>(p, dev, sms, cs, stream, pdl) : launch_mode<1, false>(p, dev, sms, cs, stream, pdl))
+                  : (fp8 ? launch_mode<0, true>(p, dev, sms, cs, stream, pdl) : launch_mode<0, false>(p, dev, sms, cs, stream, pdl));
   if (e == cudaSuccess) count_launches(1);
   return e;
 }

@@ -73,13 +73,23 @@ bool encode_bf16_map(CUtensorMap *m, const uint16_t *ptr, int64_t rows, int64_t 
 bool encode_codes_map(CUtensorMap *m, const uint8_t *ptr, int64_t rows, int64_t row_bytes, uint32_t box_bytes,
                       uint32_t box_rows, bool swizzle128);
 
+// The tensor mean of the absmax for the E4M3 + mean format (the entry after
+// the ceil(nb / 256) group scales), null for linear 8-bit.
+inline const float *mean_ptr(const float *group_scale, int64_t nblocks, int dq_format) {
+  return dq_format == kDqFp8Mean ? group_scale + (nblocks + 255) / 256 : nullptr;
+}
+
 // --- launchers (all asynchronous on `stream`; return cudaError_t) --------
 
+// dq_format is a kDq* value (types.h); for kDqFp8Mean group_scale holds
+// ceil(numel / 16384) + 1 entries, the last the tensor mean of the absmax.
 cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q,
-                            float *group_scale, float *absmax_fp32, const Nf4Tables &tab, cudaStream_t stream);
+                            float *group_scale, float *absmax_fp32, const Nf4Tables &tab, int dq_format,
+                            cudaStream_t stream);
 
 cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *absmax_q, const float *group_scale,
-                           int64_t numel, uint16_t *out, const Nf4Tables &tab, cudaStream_t stream);
+                           int64_t numel, uint16_t *out, const Nf4Tables &tab, int dq_format,
+                           cudaStream_t stream);
 
 // T[m x r] = bf16(scale * X[m x k] . A[r x k]^T) for small m (m <= 16).
 cudaError_t launch_lora_proj_small(const uint16_t *X, int64_t m, int64_t k, const uint16_t *A,
@@ -88,16 +98,16 @@ cudaError_t launch_lora_proj_small(const uint16_t *X, int64_t m, int64_t k, cons
 // Y[m x n] = bf16(X . W^T + T . B^T) for m <= 16 (CTA-ring weight-streaming
 // kernel); with pdl it overlaps the preceding T projection.
 cudaError_t launch_gemv_fwd(const uint16_t *X, int64_t m, const uint8_t *codes,
-                            const uint8_t *absmax_q, const float *group_scale, int64_t n, int64_t k,
-                            const uint16_t *T, const uint16_t *B, int32_t r, uint16_t *Y,
+                            const uint8_t *absmax_q, const float *group_scale, const float *mu, int64_t n,
+                            int64_t k, const uint16_t *T, const uint16_t *B, int32_t r, uint16_t *Y,
                             const Nf4Tables &tab, cudaStream_t stream, bool pdl);
 
 // Decode-sized forward (m <= 4, k/64 <= 512): per-warp TMA streams of the
 // codes, K split over a cluster.  Same contract as launch_gemv_fwd.
 bool gemv_stream_supported(int64_t m, int64_t n, int64_t k);
 cudaError_t launch_gemv_stream(const uint16_t *X, int64_t m, const uint8_t *codes,
-                               const uint8_t *absmax_q, const float *group_scale, int64_t n, int64_t k,
-                               const uint16_t *T, const uint16_t *B, int32_t r, uint16_t *Y,
+                               const uint8_t *absmax_q, const float *group_scale, const float *mu,
+                               int64_t n, int64_t k, const uint16_t *T, const uint16_t *B, int32_t r, uint16_t *Y,
                                const Nf4Tables &tab, cudaStream_t stream, bool pdl);
 
 // tcgen05 paths -------------------------------------------------------------
@@ -108,6 +118,7 @@ struct WeightView {
   const float *group_scale;
   int64_t n, k;
   const Nf4Tables *tab;   // the weight's codebook
+  const float *mu;        // E4M3 + mean format: the tensor mean; null for linear 8-bit
 };
 
 // Y = bf16(X . W^T + T . B^T); T may be null (no adapter).

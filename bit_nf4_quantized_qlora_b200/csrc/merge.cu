@@ -30,6 +30,7 @@ struct MergeParams {
   const uint8_t *codes;
   const uint8_t *absmax_q;
   const float *group_scale;
+  const float *mu;          // E4M3 + mean absmax format: the tensor mean; else null
   const uint16_t *A;      // [r x k]
   const uint16_t *B;      // [n x r]
   uint16_t *out_bf16;     // [n x k] or null
@@ -110,13 +111,15 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(const __grid_constant__
     cp_async16(sbase + L.codes + static_cast<uint32_t>(row) * kCodeRow + 16u * c,
                ok ? static_cast<const void *>(p.codes + ((n0 + row) * p.k + c0) / 2 + 16 * c) : p.codes, ok);
   }
-  // c' = fp32(q * fp32(S / 255)) of the tile's blocks (two per row).
+  // c' of the tile's blocks (two per row).
   {
     const int row = tid >> 1, b = tid & 1;
     float c = 0.f;
     if (n0 + row < p.n && c0 + 64 * b < p.k) {
       const int64_t blk = ((n0 + row) * p.k + c0) / 64 + b;
-      c = __fmul_rn(static_cast<float>(__ldg(p.absmax_q + blk)), div255_rn(__ldg(p.group_scale + (blk >> 8))));
+      const bool fp8 = p.mu != nullptr;
+      const float sg = __ldg(p.group_scale + (blk >> 8));
+      c = block_constant(__ldg(p.absmax_q + blk), fp8 ? sg : div255_rn(sg), fp8, load_mu(p.mu));
     }
     cp[tid] = c;
   }
@@ -232,6 +235,7 @@ cudaError_t launch_merge(const WeightView &w, const uint16_t *A, const uint16_t 
   p.codes = w.codes;
   p.absmax_q = w.absmax_q;
   p.group_scale = w.group_scale;
+  p.mu = w.mu;
   p.A = r > 0 ? A : nullptr;
   p.B = r > 0 ? B : nullptr;
   p.out_bf16 = out_bf16;

@@ -56,14 +56,45 @@ __device__ __forceinline__ uint32_t nf4_code(float x, const Nf4Tables &t) {
   return (b3 ? 8u : 0u) | (b2 ? 4u : 0u) | (b1 ? 2u : 0u) | (b0 ? 1u : 0u);
 }
 
+// Where the fp64 sum of group g's absmax values waits for the mean kernel
+// (E4M3 + mean format): in the group's own absmax-code bytes, which the final
+// pass overwrites; a partial last group (which may have fewer than 8 bytes)
+// uses bytes 8..15 of group 0 instead.  Only when there are at least two
+// groups, so group 0 is whole.
+__device__ __forceinline__ double *group_sum_slot(uint8_t *absmax_q, int64_t g, int64_t ng, bool last_partial) {
+  return reinterpret_cast<double *>(absmax_q + ((last_partial && g == ng - 1) ? 8 : 256 * g));
+}
+
+// fp64 sum of s_c[0..len) by pairwise halving (adjacent pairs, an odd last
+// element carried), the order the format fixes; every thread gets the sum.
+__device__ double group_pairwise_sum(const float *s_c, int len, double *b0, double *b1) {
+  const int t = threadIdx.x;
+  b0[t] = t < len ? static_cast<double>(s_c[t]) : 0.0;
+  __syncthreads();
+  while (len > 1) {
+    const int half = len / 2;
+    if (t < half) b1[t] = b0[2 * t] + b0[2 * t + 1];
+    if ((len & 1) && t == half) b1[half] = b0[len - 1];
+    __syncthreads();
+    double *tmp = b0;
+    b0 = b1;
+    b1 = tmp;
+    len = (len + 1) / 2;
+  }
+  const double r = b0[0];
+  __syncthreads();
+  return r;
+}
+
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const float *__restrict__ W, int64_t nb,
                                                             uint8_t *__restrict__ codes,
                                                             uint8_t *__restrict__ absmax_q,
                                                             float *__restrict__ group_scale,
                                                             float *__restrict__ absmax_out,
-                                                            const Nf4Tables tab) {
+                                                            const Nf4Tables tab, int dq_format) {
   __shared__ float s_c[kBlocksPerGroup];
   __shared__ float s_red[kThreads / 32];
+  __shared__ double s_sum[2][kBlocksPerGroup];
 
   const int64_t g = blockIdx.x;
   const int64_t b0 = g * kBlocksPerGroup;
@@ -145,6 +176,20 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const float *__restr
   }
   __syncthreads();
 
+  if (dq_format == kDqFp8Mean) {
+    // E4M3 + mean: only the group's fp64 absmax sum here; the codes of the
+    // absmax values follow once the tensor's mean is known.
+    const double sum = group_pairwise_sum(s_c, nblk, s_sum[0], s_sum[1]);
+    if (threadIdx.x == 0) {
+      const int64_t ng = gridDim.x;
+      if (ng == 1)
+        group_scale[1] = static_cast<float>(sum / static_cast<double>(nb));   // the mean itself
+      else
+        *group_sum_slot(absmax_q, g, ng, (nb % kBlocksPerGroup) != 0) = sum;
+    }
+    return;
+  }
+
   // Double quantization of this group's absmax values.
   const int t = threadIdx.x;
   const float c = (t < nblk) ? s_c[t] : 0.0f;
@@ -164,15 +209,99 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const float *__restr
   if (t == 0) group_scale[g] = S;
 }
 
+// mu = fp32(T / nb), T the pairwise sum of the ng group sums: strides 1, 2,
+// 4, ... in place (slot i += slot i + s for i a multiple of 2s), the same
+// additions as halving adjacent pairs level by level with an odd last one
+// carried.  One CTA; ng >= 2.
+__global__ void __launch_bounds__(1024) dq_mean_kernel(uint8_t *absmax_q, int64_t ng, int64_t nb,
+                                                       float *group_scale) {
+  const bool last_partial = (nb % kBlocksPerGroup) != 0;
+  for (int64_t s = 1; s < ng; s *= 2) {
+    for (int64_t i = 2 * s * threadIdx.x; i + s < ng; i += 2 * s * blockDim.x)
+      *group_sum_slot(absmax_q, i, ng, last_partial) += *group_sum_slot(absmax_q, i + s, ng, last_partial);
+    __syncthreads();
+  }
+  if (threadIdx.x == 0)
+    group_scale[ng] = static_cast<float>(*group_sum_slot(absmax_q, 0, ng, last_partial) / static_cast<double>(nb));
+}
+
+// E4M3 codes of the offsets from the mean, one CTA per group (the block
+// absmax values are recomputed from W, as in quantize_kernel):
+//   d = fp32(c - mu), S = max |d|, q = E4M3_rn(fp32(fp32(d / S) * 448)),
+//   group_scale[g] = fp32(S / 448).
+__global__ void __launch_bounds__(kThreads) dq_fp8_kernel(const float *__restrict__ W, int64_t nb,
+                                                          uint8_t *__restrict__ absmax_q,
+                                                          float *__restrict__ group_scale) {
+  __shared__ float s_red[kThreads / 32];
+  __shared__ float s_c[kBlocksPerGroup];
+  const int64_t g = blockIdx.x;
+  const int64_t b0 = g * kBlocksPerGroup;
+  const int nblk = static_cast<int>(nb - b0 < kBlocksPerGroup ? nb - b0 : kBlocksPerGroup);
+  const int64_t ng = gridDim.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane & 3, bl = lane >> 2;
+  // Block maxima with the load pattern of quantize_kernel: 4 lanes per
+  // block, each load instruction covering 8 blocks x 64 contiguous bytes.
+  float4 v[4][4];
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int blk = warp * 32 + it * 8 + bl;
+    const float4 *src = reinterpret_cast<const float4 *>(W + (b0 + blk) * 64) + sub;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[it][j] = blk < nblk ? __ldcs(src + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const float mu = __ldg(group_scale + ng);
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(v[it][j].x), fabsf(v[it][j].y)), fmaxf(fabsf(v[it][j].z), fabsf(v[it][j].w))));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    if (sub == 0) s_c[warp * 32 + it * 8 + bl] = m;
+  }
+  __syncthreads();
+  const int t = threadIdx.x;
+  const float d = t < nblk ? __fsub_rn(s_c[t], mu) : 0.f;
+  float m = fabsf(d);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) s_red[warp] = m;
+  __syncthreads();
+  float S = s_red[0];
+#pragma unroll
+  for (int i = 1; i < kThreads / 32; ++i) S = fmaxf(S, s_red[i]);
+  if (t < nblk) {
+    uint32_t q = 0;
+    if (S > 0.0f) {
+      const float x = __fmul_rn(__fdiv_rn(d, S), 448.0f);
+      uint16_t pair;
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %1;" : "=h"(pair) : "f"(x));
+      q = pair & 0xFFu;
+    }
+    absmax_q[b0 + t] = static_cast<uint8_t>(q);
+  }
+  if (t == 0) group_scale[g] = __fdiv_rn(S, 448.0f);
+}
+
 }  // namespace
 
 cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q,
-                            float *group_scale, float *absmax_fp32, const Nf4Tables &tab, cudaStream_t stream) {
+                            float *group_scale, float *absmax_fp32, const Nf4Tables &tab, int dq_format,
+                            cudaStream_t stream) {
   const int64_t nb = numel / 64;
   const int64_t ng = (nb + kBlocksPerGroup - 1) / kBlocksPerGroup;
   if (ng == 0) return cudaSuccess;
   quantize_kernel<<<static_cast<unsigned>(ng), kThreads, 0, stream>>>(W, nb, codes, absmax_q, group_scale,
-                                                                      absmax_fp32, tab);
+                                                                      absmax_fp32, tab, dq_format);
+  count_launches(1);
+  if (dq_format != kDqFp8Mean) return cudaGetLastError();
+  if (ng > 1) {
+    dq_mean_kernel<<<1, 1024, 0, stream>>>(absmax_q, ng, nb, group_scale);
+    count_launches(1);
+  }
+  dq_fp8_kernel<<<static_cast<unsigned>(ng), kThreads, 0, stream>>>(W, nb, absmax_q, group_scale);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -56,6 +56,7 @@ struct __align__(64) TcParams {
   CUtensorMap tmB2;     // adapter B operand (extra k-steps)
   const uint8_t *absmax_q;
   const float *group_scale;
+  const float *mu;                 // E4M3 + mean absmax format: the tensor mean; else null
   uint16_t *out;
   unsigned *err;
   int64_t w_n, w_k;     // weight shape (NF4 modes)
@@ -289,9 +290,12 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
         return (gn < p.w_n && kb < kblocks) ? gn * kblocks + kb : -1;
       };
       // Absmax code and group constant of this group's next step, fetched one
-      // step of the group (DQ_GROUPS k-steps) ahead.  The group constant
-      // t = fp32(S / 255) is recomputed only when the group index changes
-      // (in the forward a thread walks one weight row, so that is rare).
+      // step of the group (DQ_GROUPS k-steps) ahead.  The group constant t
+      // (fp32(S / 255) for linear codes) is recomputed only when the group
+      // index changes (in the forward a thread walks one weight row, so that
+      // is rare).
+      const bool fp8 = p.mu != nullptr;
+      const float mu = load_mu(p.mu);
       int64_t blk_nx = it_begin + grp < p.num_main ? block_of(it_begin + grp) : -1;
       uint32_t q_nx = blk_nx >= 0 ? __ldg(p.absmax_q + blk_nx) : 0u;
       float S_nx = blk_nx >= 0 ? __ldg(p.group_scale + (blk_nx >> 8)) : 0.f;
@@ -325,13 +329,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
             const int64_t gi = blk >> 8;
             if (gi != g_cur) {
               g_cur = gi;
-              t_cur = __fdiv_rn(S, 255.0f);
+              t_cur = group_constant(S, fp8);
             }
             const uint4 f = lds128(c_s + code_off + first_half);
             const uint4 g2 = lds128(c_s + code_off + (16u - first_half));
             lo = first_half ? g2 : f;
             hi = first_half ? f : g2;
-            make_table(p.tab, __fmul_rn(static_cast<float>(qv), t_cur), tb);
+            make_table(p.tab, block_constant(qv, t_cur, fp8, mu), tb);
           } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j) tb.lo[j] = tb.hi[j] = 0u;
@@ -566,6 +570,7 @@ cudaError_t tc_fwd(const uint16_t *X, int64_t m, const WeightView &w, const uint
   }
   p.absmax_q = w.absmax_q;
   p.group_scale = w.group_scale;
+  p.mu = w.mu;
   p.out = Y;
   p.err = device_error_word();
   p.w_n = w.n;
@@ -601,6 +606,7 @@ cudaError_t tc_bwd_dx(const uint16_t *dY, int64_t m, const WeightView &w, const 
   }
   p.absmax_q = w.absmax_q;
   p.group_scale = w.group_scale;
+  p.mu = w.mu;
   p.out = dX;
   p.err = device_error_word();
   p.w_n = w.n;

@@ -9,6 +9,12 @@ namespace qlora {
 // uniform-bin baselines it is compared with).
 enum : int { kCodebookNF4 = 0, kCodebookFP4 = 1, kCodebookINT4 = 2, kCodebookCount = 3 };
 
+// How the block absmax constants are stored (double quantization): unsigned
+// linear 8-bit codes with one fp32 max per group of 256, or E4M3 codes of the
+// offsets from the tensor's mean with one fp32 scale per group and the mean
+// after the group scales.
+enum : int { kDqLinear8 = 0, kDqFp8Mean = 1, kDqFormatCount = 2 };
+
 // The fp32 codebook and the 15 decision midpoints, passed by value as a
 // kernel parameter (uniform across the grid).
 struct Nf4Tables {

@@ -69,7 +69,8 @@ enum qlora_status {
   QLORA_ERR_WORKSPACE = -4, /* workspace missing or smaller than required  */
   QLORA_ERR_CUDA = -5,      /* a CUDA call failed (see last_cuda_error)    */
   QLORA_ERR_DEVICE = -6,    /* the current device is not sm_100            */
-  QLORA_ERR_CODEBOOK = -7   /* codebook id not one of qlora_codebook       */
+  QLORA_ERR_CODEBOOK = -7,  /* codebook id not one of qlora_codebook       */
+  QLORA_ERR_FORMAT = -8     /* dq_format not one of qlora_dq_format         */
 };
 
 /* The sixteen 4-bit values a weight's codes index.  NF4 is the method's own
@@ -87,6 +88,24 @@ enum qlora_status {
  * decision rule; only the levels and their midpoints change.               */
 enum qlora_codebook { QLORA_CODEBOOK_NF4 = 0, QLORA_CODEBOOK_FP4 = 1, QLORA_CODEBOOK_INT4 = 2 };
 
+/* How the block absmax constants are stored (double quantization).
+ *   QLORA_DQ_LINEAR8   unsigned linear 8-bit codes, group_scale[g] = max of
+ *                      the group's absmax (the pages' format, 0.127 bit/weight):
+ *                      c' = fp32(q * fp32(group_scale[g] / 255))
+ *   QLORA_DQ_FP8_MEAN  the cited paper's variant, which the pages name but
+ *                      do not define ("QLoRA Explained", What is QLoRA?;
+ *                      arXiv:2305.14314): the tensor's mean absmax mu is
+ *                      subtracted first and the offsets are stored as E4M3
+ *                      8-bit floats per group of 256.  mu = fp32 of the fp64
+ *                      sum of the absmax values (each group summed by
+ *                      pairwise halving, then the group sums the same way)
+ *                      over nb; S_g = max |c - mu| over the group;
+ *                      absmax_q = E4M3_rn(fp32(fp32((c - mu) / S_g) * 448));
+ *                      group_scale[g] = fp32(S_g / 448) for g < ng and
+ *                      group_scale[ng] = mu (ng + 1 floats):
+ *                      c' = fp32(fp32(E4M3(absmax_q) * group_scale[g]) + mu)  */
+enum qlora_dq_format { QLORA_DQ_LINEAR8 = 0, QLORA_DQ_FP8_MEAN = 1 };
+
 /* Quantized weight: three flat buffers plus the shape and the codebook.
  *   codes       uint8 [n*k/2]   4-bit codes, two per byte in row-major element
  *                               order: byte j = (code[2j] << 4) | code[2j+1]
@@ -95,9 +114,14 @@ enum qlora_codebook { QLORA_CODEBOOK_NF4 = 0, QLORA_CODEBOOK_FP4 = 1, QLORA_CODE
  *   block == 64 and group == 256 are the only supported values.
  *   codebook    qlora_codebook the codes index (0 == NF4, so a zeroed field
  *               means NF4); any other value gives QLORA_ERR_CODEBOOK.
+ *   dq_format   qlora_dq_format of absmax_q / group_scale (0 == linear 8-bit,
+ *               so a zeroed field means the pages' format; QLORA_DQ_FP8_MEAN
+ *               has ng + 1 group_scale entries); any other value gives
+ *               QLORA_ERR_FORMAT.
  * Dequantization ["A 65B fine-tune on the GPU you already have", figure 4;
  * "QLoRA", Storage precision is not calculation precision]:
  *   c'  = fp32(float(absmax_q[b]) * fp32(group_scale[b/256] / 255))
+ *         (QLORA_DQ_LINEAR8; the c' of QLORA_DQ_FP8_MEAN is given above)
  *   W^  = bf16_rne(fp32(L[code] * c')), L the weight's codebook            */
 typedef struct {
   const uint8_t *codes;
@@ -107,6 +131,7 @@ typedef struct {
   int32_t block;
   int32_t group;
   int32_t codebook;
+  int32_t dq_format;
 } qlora_nf4_weight;
 
 /* Operation ids for qlora_workspace_bytes. */
@@ -138,6 +163,15 @@ int qlora_quantize_nf4_dq(const float *W, int64_t n, int64_t k,
 int qlora_quantize_4bit_dq(const float *W, int64_t n, int64_t k, int32_t codebook,
                            uint8_t *codes, uint8_t *absmax_q, float *group_scale,
                            float *absmax_fp32, qlora_stream_t stream);
+
+/* The same quantization with the absmax constants stored in `dq_format`
+ * (qlora_dq_format); qlora_quantize_4bit_dq is QLORA_DQ_LINEAR8.  With
+ * QLORA_DQ_FP8_MEAN, group_scale has ng + 1 entries and the call reads W
+ * twice (the mean of all block absmax values is needed before any group's
+ * codes); absmax_q doubles as scratch between the passes.                  */
+int qlora_quantize_4bit_dq_format(const float *W, int64_t n, int64_t k, int32_t codebook, int32_t dq_format,
+                                  uint8_t *codes, uint8_t *absmax_q, float *group_scale,
+                                  float *absmax_fp32, qlora_stream_t stream);
 
 /* Standalone dequantization to bf16 ["QLoRA", Storage precision is not
  * calculation precision; "A 65B fine-tune on the GPU you already have",

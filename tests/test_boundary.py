@@ -84,14 +84,21 @@ def test_merge_rejects_bad_arguments(lib):
     assert f(ctypes.byref(_w(k=1000)), P, P, 16, 2.0, P, None, None) == B.QLORA_ERR_SHAPE
     w.codebook = 5
     assert f(ctypes.byref(w), P, P, 16, 2.0, P, None, None) == B.QLORA_ERR_CODEBOOK
+    w.codebook = 0
+    w.dq_format = 2
+    assert f(ctypes.byref(w), P, P, 16, 2.0, P, None, None) == B.QLORA_ERR_FORMAT
 
 
 def test_weight_struct_layout():
-    """Three pointers and two int64 sizes (40 bytes), then block, group and
-    codebook (int32), padded to 8 bytes: a zeroed codebook field means NF4."""
+    """Three pointers and two int64 sizes (40 bytes), then block, group,
+    codebook and dq_format (int32): 56 bytes, the size the struct had before
+    dq_format took its tail padding.  Zeroed codebook and dq_format fields
+    mean NF4 with linear 8-bit absmax codes."""
     assert ctypes.sizeof(B.NF4WeightC) == 56
     assert B.NF4WeightC.codebook.offset == 48
-    assert B.NF4WeightC(0, 0, 0, 1, 64, 64, 256).codebook == B.QLORA_CODEBOOK_NF4
+    assert B.NF4WeightC.dq_format.offset == 52
+    w = B.NF4WeightC(0, 0, 0, 1, 64, 64, 256)
+    assert w.codebook == B.QLORA_CODEBOOK_NF4 and w.dq_format == B.QLORA_DQ_LINEAR8
 
 
 def test_library_codebook_equals_oracle_codebook(lib):
@@ -103,8 +110,9 @@ def test_library_codebook_equals_oracle_codebook(lib):
 
 def test_version_and_status_strings(lib):
     assert lib.qlora_version() >> 16 == 1
-    for st in (0, -1, -2, -3, -4, -5, -6, -7):
+    for st in (0, -1, -2, -3, -4, -5, -6, -7, -8):
         assert lib.qlora_status_string(st)
+    assert b"FORMAT" in lib.qlora_status_string(B.QLORA_ERR_FORMAT)
 
 
 def test_workspace_bytes(lib):
@@ -198,6 +206,13 @@ def test_quantize_and_dequant_reject_bad_arguments(lib):
     w = _w()
     assert lib.qlora_dequant(ctypes.byref(w), None, None) == B.QLORA_ERR_NULL
     assert lib.qlora_dequant(ctypes.byref(w), MIS, None) == B.QLORA_ERR_ALIGN
+    w.dq_format = -1
+    assert lib.qlora_dequant(ctypes.byref(w), P, None) == B.QLORA_ERR_FORMAT
+    qf = lambda fmt, cb=0, W=P: lib.qlora_quantize_4bit_dq_format(W, 64, 64, cb, fmt, P, P, P, None, None)
+    assert qf(2) == B.QLORA_ERR_FORMAT
+    assert qf(-1) == B.QLORA_ERR_FORMAT
+    assert qf(B.QLORA_DQ_FP8_MEAN, cb=9) == B.QLORA_ERR_CODEBOOK
+    assert qf(B.QLORA_DQ_FP8_MEAN, W=None) == B.QLORA_ERR_NULL
     assert lib.qlora_dequant(None, P, None) == B.QLORA_ERR_NULL
 
 
