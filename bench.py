@@ -635,9 +635,39 @@ def _codebook_error(dev, reps: int = 5):
             del w, back, err
         for name in ("fp4", "int4"):
             row[name]["mse_vs_nf4"] = round(row[name]["mse"] / row["nf4"]["mse"], 3)
+        # NF4 with the absmax stored as E4M3 offsets from the mean, against the
+        # linear 8-bit format: weight round-trip error, and the error of the
+        # reconstructed block constants c' against the fp32 absmax.
+        absmax = torch.empty(W.numel() // 64, dtype=torch.float32, device=dev)
+        for fmt_name, fmt in B.DQ_FORMATS.items():
+            w = B.qlora_quantize_4bit_dq(W, B.QLORA_CODEBOOK_NF4, absmax_fp32=absmax, dq_format=fmt)
+            for _ in range(2):
+                B.qlora_quantize_4bit_dq(W, B.QLORA_CODEBOOK_NF4, absmax_fp32=absmax, out=w, dq_format=fmt)
+            torch.cuda.synchronize()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record()
+            for _ in range(reps):
+                B.qlora_quantize_4bit_dq(W, B.QLORA_CODEBOOK_NF4, out=w, dq_format=fmt)
+            t1.record()
+            torch.cuda.synchronize()
+            back = B.qlora_dequant(w).float()
+            err = back - W
+            g = torch.arange(absmax.numel(), device=dev) // 256
+            if fmt == B.QLORA_DQ_FP8_MEAN:
+                e4 = w.absmax_q.view(torch.float8_e4m3fn).float()
+                cp = (e4 * w.group_scale[g]).float() + w.group_scale[-1]
+            else:
+                cp = w.absmax_q.float() * (w.group_scale[g] / 255.0)
+            rel = (cp - absmax).abs() / absmax.clamp_min(1e-30)
+            row[f"nf4_dq_{fmt_name}"] = {"mse": float((err * err).mean()), "max_abs": float(err.abs().max()),
+                                         "absmax_rel_err_mean": float(rel.mean()),
+                                         "absmax_rel_err_max": float(rel.max()),
+                                         "quantize_us": round(t0.elapsed_time(t1) * 1e3 / reps, 1)}
+            del w, back, err, cp, rel
         out[label] = row
         del W
-    out["workload"] = "W [4096 x 4096] fp32 ~ N(0, 0.02), block 64, 8-bit double quantization per 256 blocks"
+    out["workload"] = ("W [4096 x 4096] fp32 ~ N(0, 0.02), block 64, 8-bit double quantization per 256 blocks "
+                       "(linear 8-bit codes unless the row names the E4M3 + mean format)")
     torch.cuda.empty_cache()
     return out
 
