@@ -233,7 +233,7 @@ size_t qlora_workspace_bytes(int op, int64_t m, int64_t n, int64_t k, int32_t r)
   switch (op) {
     case QLORA_OP_FWD: return r > 0 ? mr : 0;
     case QLORA_OP_BWD_DX: return r > 0 ? mr : 0;
-    case QLORA_OP_LORA_BWD: return 2 * mr;
+    case QLORA_OP_LORA_BWD: return 2 * mr + round_up(m > 0 ? dy_pass_workspace_bytes(m, n, r) : 0);
     default: return SIZE_MAX;
   }
 }
@@ -364,10 +364,14 @@ int qlora_lora_bwd(const uint16_t *X, const uint16_t *dY, int64_t m, int64_t n, 
   const size_t mr = round_up(static_cast<size_t>(m) * static_cast<size_t>(r) * 2u);
   uint16_t *T = static_cast<uint16_t *>(ws);
   uint16_t *U = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(ws) + mr);
+  void *scratch = static_cast<uint8_t *>(ws) + 2 * mr;
+  const bool one_pass = plan_dy_pass(m, n, r).ok;                         // U and dB in one pass over dY
   cudaError_t e = tc_proj_kmajor(X, m, k, A, r, scale, T, s);             // T = bf16(s X A^T)
-  if (e == cudaSuccess) e = tc_proj_mnmajor(dY, m, n, B, r, scale, U, s);  // U = bf16(s dY B)
+  if (e == cudaSuccess)
+    e = one_pass ? launch_dy_pass(dY, m, n, B, T, r, scale, U, dB, scratch, ws_bytes - 2 * mr, s, true)
+                 : tc_proj_mnmajor(dY, m, n, B, r, scale, U, s);          // U = bf16(s dY B)
   if (e == cudaSuccess) e = tc_tn_skinny(X, m, k, U, r, dA, true, s);      // dA = U^T X
-  if (e == cudaSuccess) e = tc_tn_skinny(dY, m, n, T, r, dB, false, s);    // dB = dY^T T
+  if (e == cudaSuccess && !one_pass) e = tc_tn_skinny(dY, m, n, T, r, dB, false, s);   // dB = dY^T T
   return cuda_status(e);
 }
 
@@ -401,19 +405,26 @@ int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint16_t *T, i
   const size_t mr = round_up(static_cast<size_t>(m) * static_cast<size_t>(r) * 2u);
   uint16_t *U = static_cast<uint16_t *>(ws);
   uint16_t *Tw = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(ws) + mr);
+  void *scratch = static_cast<uint8_t *>(ws) + 2 * mr;
+  const size_t scratch_bytes = ws_bytes - 2 * mr;
   // U once, for the input gradient and for dA; T from the forward when given.
+  // With r <= 64, U and dB come from one pass over dY.
+  const bool one_pass = plan_dy_pass(m, n, r).ok;
   cudaError_t e = cudaSuccess;
   if (T == nullptr) e = tc_proj_kmajor(X, m, k, A, r, scale, Tw, s);                   // T = bf16(s X A^T)
-  if (e == cudaSuccess) e = tc_proj_mnmajor(dY, m, n, B, r, scale, U, s);              // U = bf16(s dY B)
+  if (e == cudaSuccess)
+    e = one_pass ? launch_dy_pass(dY, m, n, B, T ? T : Tw, r, scale, U, dB, scratch, scratch_bytes, s,
+                                  t_prof_start == nullptr)                             // U and dB = dY^T T
+                 : tc_proj_mnmajor(dY, m, n, B, r, scale, U, s);                       // U = bf16(s dY B)
   // The input-gradient kernel needs U only for its adapter k-steps: it is
-  // launched as a programmatic dependent of the U projection, which directly
-  // precedes it (unless the caller times the main kernel alone).
+  // launched as a programmatic dependent of the kernel that writes U, which
+  // directly precedes it (unless the caller times the main kernel alone).
   const bool pdl = t_prof_start == nullptr;
   if (e == cudaSuccess) e = prof_mark(t_prof_start, s);
   if (e == cudaSuccess && dX) e = tc_bwd_dx(dY, m, view(w), U, A, r, dX, s, pdl);      // dX = dY W^ + U A
   if (e == cudaSuccess) e = prof_mark(t_prof_stop, s);
   if (e == cudaSuccess) e = tc_tn_skinny(X, m, k, U, r, dA, true, s);                  // dA = U^T X
-  if (e == cudaSuccess) e = tc_tn_skinny(dY, m, n, T ? T : Tw, r, dB, false, s);       // dB = dY^T T
+  if (e == cudaSuccess && !one_pass) e = tc_tn_skinny(dY, m, n, T ? T : Tw, r, dB, false, s);   // dB = dY^T T
   return cuda_status(e);
 }
 

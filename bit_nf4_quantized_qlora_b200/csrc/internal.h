@@ -144,6 +144,22 @@ cudaError_t tc_bwd_dx(const uint16_t *dY, int64_t m, const WeightView &w, const 
 cudaError_t tc_dropout_add(const uint16_t *U, int64_t m, int32_t r, const uint16_t *A, int64_t k,
                            const DropoutParams &d, uint16_t *dX, cudaStream_t stream);
 
+// One pass over dY for U = bf16(s dY B) [m x r] and dB = bf16(dY^T T) [n x r]
+// (r <= 64, r % 16 == 0), with fp32 partials in a scratch of
+// dy_pass_workspace_bytes (dy_pass.cu); the split depends on the shape only.
+struct DyPassPlan {
+  bool ok;
+  int nslices;           // m-slices (grid x)
+  int nranges;           // n-ranges (grid y)
+  uint32_t tmem_cols;
+  size_t upart_bytes, dpart_bytes;
+};
+DyPassPlan plan_dy_pass(int64_t m, int64_t n, int32_t r);
+size_t dy_pass_workspace_bytes(int64_t m, int64_t n, int32_t r);
+cudaError_t launch_dy_pass(const uint16_t *dY, int64_t m, int64_t n, const uint16_t *B, const uint16_t *T, int32_t r,
+                           float scale, uint16_t *U, uint16_t *dB, void *scratch, size_t scratch_bytes,
+                           cudaStream_t stream, bool pdl_reduce);
+
 // Adapter merge W' = W^ + scale * B . A (B [n x r], A [r x k], r % 16 == 0,
 // r <= 256; r == 0 gives W^), written as bf16 and/or fp32 [n x k].
 cudaError_t launch_merge(const WeightView &w, const uint16_t *A, const uint16_t *B, int32_t r, float scale,

@@ -238,7 +238,10 @@ int qlora_linear_bwd_dx(const uint16_t *dY, int64_t m, const qlora_nf4_weight *w
  *   A, B   in   bf16 [r x k], [n x r], r > 0
  *   dA, dB out  bf16; overwritten (not accumulated)
  *   ws     scratch, ws_bytes >= qlora_workspace_bytes(QLORA_OP_LORA_BWD, m, n, k, r)
- * m == 0 writes zeros to dA and dB.                                        */
+ * m == 0 writes zeros to dA and dB.  For r <= 64, U = bf16(s . dY . B) and
+ * dB come from one read of dY (one kernel forms both products, then a small
+ * kernel adds the fp32 partials of U in a fixed order); results do not
+ * depend on the launch configuration's timing (no atomics).                */
 int qlora_lora_bwd(const uint16_t *X, const uint16_t *dY, int64_t m, int64_t n, int64_t k,
                    const uint16_t *A, const uint16_t *B, int32_t r, float scale,
                    uint16_t *dA, uint16_t *dB, void *ws, size_t ws_bytes,
@@ -256,7 +259,8 @@ int qlora_lora_bwd(const uint16_t *X, const uint16_t *dY, int64_t m, int64_t n, 
  *   dY, X  in   bf16 [m x n], [m x k];  A, B as in the forward, r > 0
  *   dX, dA, dB out  (dX may be NULL); ws >= qlora_workspace_bytes(QLORA_OP_LORA_BWD, m, n, k, r)
  * m == 0 writes zeros to dA and dB.  Same results as qlora_linear_bwd_dx
- * followed by qlora_lora_bwd, with two fewer rank-r projections.           */
+ * followed by qlora_lora_bwd, with two fewer rank-r projections; for r <= 64
+ * U and dB share one read of dY, as in qlora_lora_bwd.                     */
 int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const uint16_t *T, int64_t m,
                      const qlora_nf4_weight *w, const uint16_t *A, const uint16_t *B, int32_t r,
                      float scale, uint16_t *dX, uint16_t *dA, uint16_t *dB, void *ws, size_t ws_bytes,
@@ -324,7 +328,11 @@ int qlora_linear_fwd_noalloc(const uint16_t *X, int64_t m, const qlora_nf4_weigh
 
 /* Workspace bytes an operation needs (0 if none); SIZE_MAX for an unknown op
  * or invalid sizes.  A workspace may be reused across calls on one stream;
- * two calls that may run concurrently need separate workspaces.             */
+ * two calls that may run concurrently need separate workspaces.
+ * QLORA_OP_LORA_BWD (also qlora_linear_bwd): U and T ([m x r] bf16 each,
+ * 256-byte aligned), then for r <= 64 the fp32 partials of U, one [m x r]
+ * block per n-range of the one-pass kernel (at most one range per 128
+ * columns of n; the bound holds for any device).                           */
 size_t qlora_workspace_bytes(int op, int64_t m, int64_t n, int64_t k, int32_t r);
 
 /* cudaError_t of the last failing CUDA call on this host thread (0 if none). */

@@ -121,7 +121,13 @@ def test_workspace_bytes(lib):
     assert f(B.QLORA_OP_FWD, 4096, 11008, 4096, 64) == 4096 * 64 * 2
     assert f(B.QLORA_OP_FWD, 3, 1024, 1024, 16) == 256          # rounded up to 256 B
     assert f(B.QLORA_OP_BWD_DX, 16, 1024, 1024, 16) == 512
-    assert f(B.QLORA_OP_LORA_BWD, 16, 1024, 1024, 16) == 1024
+    # U and T (2 x 512 B), then the fp32 partials of the one-pass adapter
+    # products for r <= 64: U of each n-range (here 8 ranges of one 128-column
+    # block: the split that gives the busiest CTA the fewest stages) and dB of
+    # each m-slice (one: m fits one 128-row block).
+    assert f(B.QLORA_OP_LORA_BWD, 16, 1024, 1024, 16) == 1024 + 8 * 16 * 16 * 4 + 1 * 1024 * 16 * 4
+    # r > 64 keeps the separate products: U and T only.
+    assert f(B.QLORA_OP_LORA_BWD, 16, 1024, 1024, 128) == 2 * 16 * 128 * 2
     assert f(99, 1, 1, 1, 1) == 2 ** 64 - 1
     assert f(B.QLORA_OP_FWD, -1, 1, 1, 1) == 2 ** 64 - 1
 
