@@ -263,7 +263,7 @@ int qlora_quantize_4bit_dq_format(const float *W, int64_t n, int64_t k, int32_t 
   int st = check_device();
   if (st != QLORA_OK) return st;
   return cuda_status(launch_quantize(W, n * k, codes, absmax_q, group_scale, absmax_fp32, codebook_tables(codebook),
-                                     dq_format, reinterpret_cast<cudaStream_t>(stream)));
+                                     codebook_buckets(codebook), dq_format, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int qlora_merge_adapter(const qlora_nf4_weight *w, const uint16_t *A, const uint16_t *B, int32_t r, float scale,

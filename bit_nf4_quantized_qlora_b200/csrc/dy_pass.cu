@@ -60,8 +60,9 @@ struct __align__(64) PassParams {
   CUtensorMap tmDY;    // dY [m x n], box {64, 128}
   CUtensorMap tmB;     // B  [n x r], box {64, 128}
   CUtensorMap tmT;     // T  [m x r], box {64, 128}
+  CUtensorMap tmD;     // dB partials [S][n][r] fp32, box {32, 128, 1}
   float *upart;        // [R x m x r] fp32: U of each n-range
-  float *dpart;        // [S x n x r] fp32: dB of each m-slice
+  float *dpart;        // [S x n x r] fp32: dB of each m-slice (written through tmD)
   unsigned *err;
   int m, n, r;
   int mblocks, nblocks;
@@ -77,6 +78,13 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
         "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(z), "r"(src)
+               : "memory");
 }
 
 // Balanced split of `total` items into `parts`: the first item of part i.
@@ -232,6 +240,10 @@ __global__ void __launch_bounds__(kThreads, 1) dy_pass_kernel(const __grid_const
   }
 
   // ------------------------------------------------------------ dB partials
+  // Each n-block's [128 x r] fp32 partial goes through shared memory (the
+  // ring is free once every MMA has completed) as 128-byte-swizzled boxes of
+  // 32 columns, written out by TMA stores (rows past n are clipped).
+  const int nbox = (p.r + 31) / 32;
   if (warp >= 2) {
     const bool acc_ok = nmb == 0 || mbar_wait_bounded(dbfull, 0u, p.err, kErrTimeoutAcc, 20000000000ull);
     tc_fence_after();
@@ -239,8 +251,6 @@ __global__ void __launch_bounds__(kThreads, 1) dy_pass_kernel(const __grid_const
     const int row = q * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
     for (int j = 0; j < nnb; ++j) {
-      const int nrow = (nb0 + j) * 128 + row;
-      float *dst = p.dpart + (static_cast<int64_t>(slice) * p.n + nrow) * p.r;
       for (int c = 0; c < p.r; c += 16) {
         uint32_t v[16];
         if (nmb > 0 && acc_ok) {
@@ -249,15 +259,23 @@ __global__ void __launch_bounds__(kThreads, 1) dy_pass_kernel(const __grid_const
 #pragma unroll
           for (int e = 0; e < 16; ++e) v[e] = 0u;
         }
-        if (nrow < p.n) {
-          float4 *d4 = reinterpret_cast<float4 *>(dst + c);
+        const uint32_t box = base + static_cast<uint32_t>(j * 2 + c / 32) * kBox;
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            d4[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t chunk = static_cast<uint32_t>((c % 32) / 4 + e);
+          const uint32_t w[4] = {v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]};
+          sts128(box + row * 128u + ((chunk ^ static_cast<uint32_t>(row & 7)) << 4), w);
         }
       }
     }
+    fence_proxy_async_smem();
+  }
+  __syncthreads();
+  if (warp == 2 && lane == 0) {
+    for (int j = 0; j < nnb; ++j)
+      for (int b = 0; b < nbox; ++b)
+        tma_store_3d(&p.tmD, base + static_cast<uint32_t>(j * 2 + b) * kBox, 32 * b, (nb0 + j) * 128, slice);
+    tma_store_drain();
   }
   tc_fence_before();
   __syncthreads();
@@ -368,6 +386,7 @@ cudaError_t launch_dy_pass(const uint16_t *dY, int64_t m, int64_t n, const uint1
   if (!encode_bf16_map(&p.tmDY, dY, m, n, 64, 128)) return cudaErrorInvalidValue;
   if (!encode_bf16_map(&p.tmB, B, n, r, 64, 128)) return cudaErrorInvalidValue;
   if (!encode_bf16_map(&p.tmT, T, m, r, 64, 128)) return cudaErrorInvalidValue;
+  if (!encode_f32_slab_map(&p.tmD, dpart, pl.nslices, n, r, 32, 128)) return cudaErrorInvalidValue;
   p.upart = upart;
   p.dpart = dpart;
   p.err = device_error_word();

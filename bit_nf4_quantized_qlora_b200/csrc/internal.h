@@ -18,6 +18,7 @@ constexpr int kMaxDevicesPerProcess = 64;
 // The library's codebooks and their midpoints (derived once at load time):
 // codebook_tables(kCodebookNF4 | kCodebookFP4 | kCodebookINT4).
 const Nf4Tables &codebook_tables(int codebook);
+const QuantBuckets &codebook_buckets(int codebook);
 const Nf4Tables &nf4_tables();
 
 // Device error word (bounded waits that gave up); one per device.
@@ -70,6 +71,11 @@ cudaError_t launch_dropout_apply(const uint16_t *X, int64_t numel, const Dropout
 // rows of packed codes, optional 128-byte swizzle.  False if encoding failed.
 bool encode_bf16_map(CUtensorMap *m, const uint16_t *ptr, int64_t rows, int64_t cols, uint32_t box_cols,
                      uint32_t box_rows);
+// 3D map over `slabs` row-major fp32 [rows x cols] matrices; 128-byte
+// swizzled boxes of {box_cols (<= 32), box_rows, 1}.  Stores clip at the
+// slab's rows and columns.
+bool encode_f32_slab_map(CUtensorMap *m, const float *ptr, int64_t slabs, int64_t rows, int64_t cols,
+                         uint32_t box_cols, uint32_t box_rows);
 bool encode_codes_map(CUtensorMap *m, const uint8_t *ptr, int64_t rows, int64_t row_bytes, uint32_t box_bytes,
                       uint32_t box_rows, bool swizzle128);
 
@@ -84,8 +90,8 @@ inline const float *mean_ptr(const float *group_scale, int64_t nblocks, int dq_f
 // dq_format is a kDq* value (types.h); for kDqFp8Mean group_scale holds
 // ceil(numel / 16384) + 1 entries, the last the tensor mean of the absmax.
 cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q,
-                            float *group_scale, float *absmax_fp32, const Nf4Tables &tab, int dq_format,
-                            cudaStream_t stream);
+                            float *group_scale, float *absmax_fp32, const Nf4Tables &tab, const QuantBuckets &bk,
+                            int dq_format, cudaStream_t stream);
 
 cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *absmax_q, const float *group_scale,
                            int64_t numel, uint16_t *out, const Nf4Tables &tab, int dq_format,

@@ -26,6 +26,8 @@
 // Midpoints as for NF4: fp32(L_i + L_i+1) halved.
 #include <algorithm>
 #include <cmath>
+#include <cstring>
+#include <limits>
 #include <mutex>
 
 #include "internal.h"
@@ -100,12 +102,45 @@ Nf4Tables with_midpoints(Nf4Tables t) {
   return t;
 }
 
+// Bucket tables of a codebook for the quantizer (see QuantBuckets).
+QuantBuckets build_buckets(const Nf4Tables &t) {
+  QuantBuckets q{};
+  int bucket_of[15];
+  for (int i = 0; i < 15; ++i) {
+    // The device's rn(15.4 x + 16): one fp32 FMA with 1.5 * 2^23 + 16.
+    const float u = std::fmaf(t.mid[i], 15.4f, 12582928.0f);
+    uint32_t bits;
+    std::memcpy(&bits, &u, 4);
+    const int b = static_cast<int>(bits - 0x4B400000u);
+    bucket_of[i] = b < 0 ? 0 : (b > 31 ? 31 : b);
+    if (t.mid[i] == 0.0f) q.zero_mid = 1;
+  }
+  q.ok = 1;
+  for (int b = 0; b < 32; ++b) {
+    int c = 0;
+    while (c < 15 && bucket_of[c] < b) ++c;
+    q.code[b] = static_cast<uint32_t>(c);
+    q.thr[b] = c < 15 ? t.mid[c] : std::numeric_limits<float>::infinity();
+    // A second midpoint in this bucket must be out of reach of |x| <= 1.
+    for (int i = c + 1; i < 15 && bucket_of[i] == b; ++i)
+      if (t.mid[i] < 1.0f) q.ok = 0;
+  }
+  return q;
+}
+
 }  // namespace
 
 const Nf4Tables &codebook_tables(int codebook) {
   static const Nf4Tables tables[kCodebookCount] = {with_midpoints(build_tables()), with_midpoints(build_fp4()),
                                                    with_midpoints(build_int4())};
   return tables[(codebook >= 0 && codebook < kCodebookCount) ? codebook : kCodebookNF4];
+}
+
+const QuantBuckets &codebook_buckets(int codebook) {
+  static const QuantBuckets b[kCodebookCount] = {build_buckets(codebook_tables(kCodebookNF4)),
+                                                 build_buckets(codebook_tables(kCodebookFP4)),
+                                                 build_buckets(codebook_tables(kCodebookINT4))};
+  return b[(codebook >= 0 && codebook < kCodebookCount) ? codebook : kCodebookNF4];
 }
 
 const Nf4Tables &nf4_tables() { return codebook_tables(kCodebookNF4); }

@@ -31,15 +31,16 @@ constexpr int kBlocksPerGroup = 256;
 // separately in div_by_absmax.)
 constexpr float kMinFastAbsmax = 0x1p-90f;
 
+template <bool TINY>
 __device__ __forceinline__ float div_by_absmax(float w, float m, float y) {
   const float q0 = __fmul_rn(w, y);
   const float rho = __fmaf_rn(-q0, m, w);
   float x = __fmaf_rn(rho, y, q0);
   // Below the normal range the residual can underflow and the result may be
   // off by an ulp.  Only zero against nonzero (and the sign) can decide a
-  // code there, and only in a codebook with a midpoint at 0 (FP4: -0 | +0):
-  // IEEE division settles those rare quotients.
-  if (fabsf(x) < 0x1p-125f) x = __fdiv_rn(w, m);
+  // code there, and only in a codebook with a midpoint at 0 (TINY, FP4:
+  // -0 | +0): IEEE division settles those rare quotients.
+  if (TINY && fabsf(x) < 0x1p-125f) x = __fdiv_rn(w, m);
   return x;
 }
 
@@ -54,6 +55,18 @@ __device__ __forceinline__ uint32_t nf4_code(float x, const Nf4Tables &t) {
   const float hi = b1 ? (b3 ? t.mid[14] : t.mid[6]) : (b3 ? t.mid[12] : t.mid[4]);
   const bool b0 = x > (b2 ? hi : lo);
   return (b3 ? 8u : 0u) | (b2 ? 4u : 0u) | (b1 ? 2u : 0u) | (b0 ? 1u : 0u);
+}
+
+// The same count by bucket (QuantBuckets): one FMA, two shuffles from the
+// lane-held tables (lane b holds code[b] and thr[b]) and one compare.  All
+// lanes of the warp take part.
+__device__ __forceinline__ uint32_t bucket_code(float x, uint32_t lane_code, float lane_thr) {
+  // u = 1.5 * 2^23 + rn(15.4 x + 16): the bucket is the low five bits of u,
+  // which is all a shuffle takes of its source lane.
+  const int u = __float_as_int(__fmaf_rn(x, 15.4f, 12582928.0f));
+  const uint32_t c = __shfl_sync(0xffffffffu, lane_code, u);
+  const float t = __shfl_sync(0xffffffffu, lane_thr, u);
+  return c + (x > t ? 1u : 0u);
 }
 
 // Where the fp64 sum of group g's absmax values waits for the mean kernel
@@ -86,12 +99,16 @@ __device__ double group_pairwise_sum(const float *s_c, int len, double *b0, doub
   return r;
 }
 
+// BUCKET: codes by bucket_code (codebooks whose buckets allow it), else by
+// the binary search.  TINY: the codebook has a midpoint at 0.
+template <bool BUCKET, bool TINY>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const float *__restrict__ W, int64_t nb,
                                                             uint8_t *__restrict__ codes,
                                                             uint8_t *__restrict__ absmax_q,
                                                             float *__restrict__ group_scale,
                                                             float *__restrict__ absmax_out,
-                                                            const Nf4Tables tab, int dq_format) {
+                                                            const Nf4Tables tab, const QuantBuckets bk,
+                                                            int dq_format) {
   __shared__ float s_c[kBlocksPerGroup];
   __shared__ float s_red[kThreads / 32];
   __shared__ double s_sum[2][kBlocksPerGroup];
@@ -103,6 +120,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const float *__restr
   const int lane = threadIdx.x & 31;
   const int sub = lane & 3;      // 4 lanes per block, 16 weights each
   const int bl = lane >> 2;      // 8 blocks per warp iteration
+  const uint32_t lane_code = BUCKET ? bk.code[lane] : 0u;
+  const float lane_thr = BUCKET ? bk.thr[lane] : 0.f;
 
   // Warp w owns blocks [32w, 32w + 32): 4 iterations of 8 blocks.  Lane
   // (bl, sub) holds weights 16j + 4sub .. +3 (j = 0..3) of its block, so each
@@ -130,39 +149,45 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const float *__restr
       m = fmaxf(m, fmaxf(fmaxf(fabsf(v[j].x), fabsf(v[j].y)), fmaxf(fabsf(v[j].z), fabsf(v[j].w))));
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    if (blk < nblk) {
-      uint32_t c[16];
-      if (m >= kMinFastAbsmax) {
-        // Correctly rounded w / m without a divide per weight (Markstein's
-        // theorem): with y = RN(1/m) and q0 = RN(w*y) within one ulp of w/m,
-        // the residual w - m*q0 is exact in one FMA and RN(q0 + residual*y)
-        // is RN(w/m).  |w/m| <= 1 cannot overflow; results below the normal
-        // range are redone by IEEE division (div_by_absmax).
-        const float y = __frcp_rn(m);
+    // Quotients x = fp32(w / m) (per-lane branches, no shuffles inside).
+    float x[16];
+    if (m >= kMinFastAbsmax) {
+      // Correctly rounded w / m without a divide per weight (Markstein's
+      // theorem): with y = RN(1/m) and q0 = RN(w*y) within one ulp of w/m,
+      // the residual w - m*q0 is exact in one FMA and RN(q0 + residual*y)
+      // is RN(w/m).  |w/m| <= 1 cannot overflow; results below the normal
+      // range are redone by IEEE division (div_by_absmax).
+      const float y = __frcp_rn(m);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          c[4 * j + 0] = nf4_code(div_by_absmax(v[j].x, m, y), tab);
-          c[4 * j + 1] = nf4_code(div_by_absmax(v[j].y, m, y), tab);
-          c[4 * j + 2] = nf4_code(div_by_absmax(v[j].z, m, y), tab);
-          c[4 * j + 3] = nf4_code(div_by_absmax(v[j].w, m, y), tab);
-        }
-      } else if (m > 0.0f) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          c[4 * j + 0] = nf4_code(__fdiv_rn(v[j].x, m), tab);
-          c[4 * j + 1] = nf4_code(__fdiv_rn(v[j].y, m), tab);
-          c[4 * j + 2] = nf4_code(__fdiv_rn(v[j].z, m), tab);
-          c[4 * j + 3] = nf4_code(__fdiv_rn(v[j].w, m), tab);
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) c[e] = 7u;
+      for (int j = 0; j < 4; ++j) {
+        x[4 * j + 0] = div_by_absmax<TINY>(v[j].x, m, y);
+        x[4 * j + 1] = div_by_absmax<TINY>(v[j].y, m, y);
+        x[4 * j + 2] = div_by_absmax<TINY>(v[j].z, m, y);
+        x[4 * j + 3] = div_by_absmax<TINY>(v[j].w, m, y);
       }
+    } else if (m > 0.0f) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        x[4 * j + 0] = __fdiv_rn(v[j].x, m);
+        x[4 * j + 1] = __fdiv_rn(v[j].y, m);
+        x[4 * j + 2] = __fdiv_rn(v[j].z, m);
+        x[4 * j + 3] = __fdiv_rn(v[j].w, m);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) x[e] = 0.f;
+    }
+    // Codes (the warp converged again: bucket_code shuffles).  A zero block
+    // takes code 7.
+    uint32_t c[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) c[e] = BUCKET ? bucket_code(x[e], lane_code, lane_thr) : nf4_code(x[e], tab);
+    if (blk < nblk) {
       uint16_t *dst = reinterpret_cast<uint16_t *>(codes + (b0 + blk) * 32);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const uint32_t packed = ((c[4 * j] << 4) | c[4 * j + 1]) | (((c[4 * j + 2] << 4) | c[4 * j + 3]) << 8);
-        dst[4 * j + sub] = static_cast<uint16_t>(packed);      // bytes 8j + 2sub, +1
+        dst[4 * j + sub] = static_cast<uint16_t>(m > 0.0f ? packed : 0x7777u);   // bytes 8j + 2sub, +1
       }
       if (sub == 0) {
         s_c[blk] = m;
@@ -288,13 +313,21 @@ __global__ void __launch_bounds__(kThreads) dq_fp8_kernel(const float *__restric
 }  // namespace
 
 cudaError_t launch_quantize(const float *W, int64_t numel, uint8_t *codes, uint8_t *absmax_q,
-                            float *group_scale, float *absmax_fp32, const Nf4Tables &tab, int dq_format,
-                            cudaStream_t stream) {
+                            float *group_scale, float *absmax_fp32, const Nf4Tables &tab, const QuantBuckets &bk,
+                            int dq_format, cudaStream_t stream) {
   const int64_t nb = numel / 64;
   const int64_t ng = (nb + kBlocksPerGroup - 1) / kBlocksPerGroup;
   if (ng == 0) return cudaSuccess;
-  quantize_kernel<<<static_cast<unsigned>(ng), kThreads, 0, stream>>>(W, nb, codes, absmax_q, group_scale,
-                                                                      absmax_fp32, tab, dq_format);
+  const dim3 grid(static_cast<unsigned>(ng));
+  if (bk.ok && !bk.zero_mid)
+    quantize_kernel<true, false><<<grid, kThreads, 0, stream>>>(W, nb, codes, absmax_q, group_scale, absmax_fp32, tab,
+                                                               bk, dq_format);
+  else if (bk.ok)
+    quantize_kernel<true, true><<<grid, kThreads, 0, stream>>>(W, nb, codes, absmax_q, group_scale, absmax_fp32, tab,
+                                                              bk, dq_format);
+  else
+    quantize_kernel<false, true><<<grid, kThreads, 0, stream>>>(W, nb, codes, absmax_q, group_scale, absmax_fp32, tab,
+                                                               bk, dq_format);
   count_launches(1);
   if (dq_format != kDqFp8Mean) return cudaGetLastError();
   if (ng > 1) {

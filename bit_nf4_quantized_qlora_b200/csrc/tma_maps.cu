@@ -42,6 +42,19 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint64_t 
 
 }  // namespace
 
+bool encode_f32_slab_map(CUtensorMap *m, const float *ptr, int64_t slabs, int64_t rows, int64_t cols,
+                         uint32_t box_cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slabs)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 4u, static_cast<cuuint64_t>(rows * cols) * 4u};
+  cuuint32_t box[3] = {box_cols, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_bf16_map(CUtensorMap *m, const uint16_t *ptr, int64_t rows, int64_t cols, uint32_t box_cols,
                      uint32_t box_rows) {
   return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, static_cast<uint64_t>(cols), static_cast<uint64_t>(rows),

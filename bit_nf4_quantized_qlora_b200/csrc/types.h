@@ -23,6 +23,22 @@ struct Nf4Tables {
   float pad_;
 };
 
+// The code of a quotient x in [-1, 1] by bucket: b = rn(15.4 x + 16), in
+// [1, 31] (one fp32 FMA with the 1.5 * 2^23 rounding constant: b is the low
+// bits of the result), then code = code[b] + (x > thr[b]), with code[b] the
+// number of midpoints in lower buckets and thr[b] the next midpoint (+inf
+// past the last).  The bucket index is monotone in x, so a midpoint in a
+// lower bucket is below x and one in a higher bucket above it; this is exact
+// when no bucket holds a second midpoint that some |x| <= 1 can exceed
+// (ok == 1).  zero_mid: a midpoint is exactly 0, so the sign of a quotient
+// below the normal range decides a code.
+struct QuantBuckets {
+  uint32_t code[32];
+  float thr[32];
+  int32_t ok;
+  int32_t zero_mid;
+};
+
 // Device-side error codes written to the caller-visible error word when a
 // bounded wait gives up (no kernel ever traps).
 enum : unsigned {
