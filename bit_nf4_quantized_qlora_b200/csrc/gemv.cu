@@ -307,9 +307,16 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
     const int nl = r_lo + (i % rpr);
     const int64_t n = n_cta + nl;
     if (n >= p.n) continue;
-    float sum = 0.f;
     const uint32_t off = red_addr + static_cast<uint32_t>(mi * kRows + nl) * 4u;
-    for (uint32_t peer = 0; peer < csize; ++peer) sum += ld_dsmem_f32(off, peer);
+    // Every peer's partial is requested before the first add (a cluster has
+    // at most 8 CTAs); the adds run in peer order.
+    float part[8];
+#pragma unroll
+    for (uint32_t peer = 0; peer < 8; ++peer) part[peer] = peer < csize ? ld_dsmem_f32(off, peer) : 0.f;
+    float sum = 0.f;
+#pragma unroll
+    for (uint32_t peer = 0; peer < 8; ++peer)
+      if (peer < csize) sum += part[peer];
     if (p.r > 0) {
       const uint16_t *trow = p.T + static_cast<int64_t>(mi) * p.r;
       const uint16_t *brow = p.B + n * p.r;

@@ -427,8 +427,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const __grid_c
     const int64_t n = static_cast<int64_t>(t_lo + ut) * kTileRows + rl;
     if (n >= p.n) continue;
     const uint32_t off = red_addr + static_cast<uint32_t>((ut * kMaxM + mi) * kTileRows + rl) * 4u;
+    // Every peer's partial is requested before the first add; the adds run
+    // in peer order.
+    float part[kMaxCluster];
+#pragma unroll
+    for (uint32_t peer = 0; peer < kMaxCluster; ++peer) part[peer] = peer < csize ? ld_dsmem_f32(off, peer) : 0.f;
     float sum = 0.f;
-    for (uint32_t peer = 0; peer < csize; ++peer) sum += ld_dsmem_f32(off, peer);
+#pragma unroll
+    for (uint32_t peer = 0; peer < kMaxCluster; ++peer)
+      if (peer < csize) sum += part[peer];
     if (p.r > 0) {
       const uint16_t *trow = p.T + static_cast<int64_t>(mi) * p.r;
       const uint16_t *brow = p.B + n * p.r;

@@ -113,8 +113,12 @@ struct Cfg {
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
   static_assert(!SPLIT || (MSUB == 1 && (B_NF4 ? BN == 256 : BN == 64)),
                 "split-K: the skinny products and the small-M NF4 products");
-  static_assert(!SPLIT || STAGE_BYTES * STAGES >= 128u * static_cast<uint32_t>(BN) * 4u,
-                "room for the fp32 partial tile");
+  // Split-K partial tile, laid out along the output's contiguous dimension:
+  // row-major with rows of BN fp32 padded by 16 bytes (the 16-byte pieces of
+  // 8 consecutive rows land in 8 distinct bank groups) for a row-major
+  // output, column-major (128 fp32 per column) for a transposed one.
+  static constexpr uint32_t PART_LD = static_cast<uint32_t>(BN) + 4u;
+  static_assert(!SPLIT || STAGE_BYTES * STAGES >= 128u * PART_LD * 4u, "room for the fp32 partial tile");
   static_assert(EPI == kEpiStore || (!SPLIT && !OUT_T && !B_NF4), "masked add: plain row-major output");
 };
 
@@ -388,12 +392,24 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
         uint32_t v[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(h * C::BN + c0), v);
         if (C::SPLIT) {
-          // fp32 partial, column-major [col][row] in this CTA's idle stage memory.
-          const uint32_t dst = base + (static_cast<uint32_t>(c0) * 128u + static_cast<uint32_t>(row_in_tile)) * 4u;
+          // fp32 partial in this CTA's idle stage memory.
+          if (!C::OUT_T) {
+            const uint32_t dst =
+                base + (static_cast<uint32_t>(row_in_tile) * C::PART_LD + static_cast<uint32_t>(c0)) * 4u;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float val = n_iters > 0 ? __uint_as_float(v[j]) : 0.f;
-            asm volatile("st.shared.f32 [%0], %1;" ::"r"(dst + static_cast<uint32_t>(j) * 512u), "f"(val) : "memory");
+            for (int j = 0; j < 8; ++j) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) w[e] = n_iters > 0 ? v[4 * j + e] : 0u;
+              sts128(dst + 16u * static_cast<uint32_t>(j), w);
+            }
+          } else {
+            const uint32_t dst = base + (static_cast<uint32_t>(c0) * 128u + static_cast<uint32_t>(row_in_tile)) * 4u;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float val = n_iters > 0 ? __uint_as_float(v[j]) : 0.f;
+              asm volatile("st.shared.f32 [%0], %1;" ::"r"(dst + static_cast<uint32_t>(j) * 512u), "f"(val) : "memory");
+            }
           }
           continue;
         }
@@ -459,25 +475,91 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) tc_kernel(const __grid_cons
   __syncthreads();
   if (C::SPLIT) {
     // Reduce the cluster's partial tiles through distributed shared memory:
-    // CTA `rank` finishes rows [rank*v/size, (rank+1)*v/size) of the tile's
-    // v rows that exist in the output.
+    // CTA `rank` finishes a share of the tile's rows that exist in the output
+    // (in whole groups of four rows for a transposed output).
     cluster_sync_all();
     const uint32_t rank = cluster_rank(), size = cluster_size();
     const int64_t left = static_cast<int64_t>(p.out_rows) - static_cast<int64_t>(m_tile) * C::BM;
     const uint32_t valid = static_cast<uint32_t>(left < 128 ? (left > 0 ? left : 0) : 128);
-    const int r_lo = static_cast<int>((valid * rank) / size), r_hi = static_cast<int>((valid * (rank + 1)) / size);
-    const int rows = r_hi - r_lo;
-    for (int i = threadIdx.x; i < rows * C::BN; i += C::NUM_THREADS) {
-      const int col = i / rows, row = r_lo + (i % rows);
-      const uint32_t off = base + (static_cast<uint32_t>(col) * 128u + static_cast<uint32_t>(row)) * 4u;
-      float acc = 0.f;
-      for (uint32_t pr = 0; pr < size; ++pr) acc += ld_dsmem_f32(off, pr);
-      const int64_t grow = static_cast<int64_t>(m_tile) * C::BM + row;
-      const int64_t gcol = static_cast<int64_t>(n_tile) * C::BN + col;
-      if (grow < p.out_rows && gcol < p.out_cols) {
-        const uint16_t v = static_cast<uint16_t>(pack_bf16x2(acc * p.alpha, 0.f) & 0xFFFFu);
-        if (C::OUT_T) p.out[gcol * p.out_ld + grow] = v;
-        else p.out[grow * p.out_ld + gcol] = v;
+    const uint32_t units = C::OUT_T ? (valid + 3u) / 4u : valid;
+    const int u_lo = static_cast<int>((units * rank) / size), u_hi = static_cast<int>((units * (rank + 1)) / size);
+    const int nu = u_hi - u_lo;
+    // Work items are 16-byte pieces along the partial's contiguous dimension:
+    // (row, 4 columns) for a row-major output, (column, 4 rows) for a
+    // transposed one; consecutive threads take consecutive pieces, so the
+    // remote reads and the bf16 stores are contiguous.  A thread takes kBatch
+    // pieces at a time and issues all their peer loads (up to 8 peers) before
+    // the first add, so the remote-load latency is paid once per batch; each
+    // piece's partials are added in peer order.
+    constexpr int kBatch = C::NUM_THREADS > 256 ? 1 : 2;   // 32 registers of partials per piece
+    constexpr int kPieces = C::BN / 4;                      // pieces per row (row-major output)
+    const int nel = C::OUT_T ? nu * C::BN : nu * kPieces;
+    const bool vec_ok = (p.out_ld & 3) == 0 && (reinterpret_cast<uintptr_t>(p.out) & 7u) == 0;
+    for (int i0 = threadIdx.x; i0 < nel; i0 += kBatch * C::NUM_THREADS) {
+      float4 part[kBatch][8];
+      int row[kBatch], col[kBatch];
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        const int i = i0 + b * C::NUM_THREADS;
+        const bool live = i < nel;
+        const int ii = live ? i : 0;
+        uint32_t off;
+        if (!C::OUT_T) {
+          row[b] = u_lo + ii / kPieces;
+          col[b] = 4 * (ii % kPieces);
+          off = base + (static_cast<uint32_t>(row[b]) * C::PART_LD + static_cast<uint32_t>(col[b])) * 4u;
+        } else {
+          row[b] = 4 * (u_lo + ii % nu);
+          col[b] = ii / nu;
+          off = base + (static_cast<uint32_t>(col[b]) * 128u + static_cast<uint32_t>(row[b])) * 4u;
+        }
+        if (!live) col[b] = -1;
+#pragma unroll
+        for (int pr = 0; pr < 8; ++pr)
+          part[b][pr] = (live && static_cast<uint32_t>(pr) < size) ? ld_dsmem_v4(off, static_cast<uint32_t>(pr))
+                                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        if (col[b] < 0) continue;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int pr = 0; pr < 8; ++pr) {
+          if (static_cast<uint32_t>(pr) < size) {
+            acc.x += part[b][pr].x;
+            acc.y += part[b][pr].y;
+            acc.z += part[b][pr].z;
+            acc.w += part[b][pr].w;
+          }
+        }
+        const int64_t grow = static_cast<int64_t>(m_tile) * C::BM + row[b];
+        const int64_t gcol = static_cast<int64_t>(n_tile) * C::BN + col[b];
+        const uint32_t h01 = pack_bf16x2(acc.x * p.alpha, acc.y * p.alpha);
+        const uint32_t h23 = pack_bf16x2(acc.z * p.alpha, acc.w * p.alpha);
+        const uint16_t h[4] = {static_cast<uint16_t>(h01 & 0xFFFFu), static_cast<uint16_t>(h01 >> 16),
+                               static_cast<uint16_t>(h23 & 0xFFFFu), static_cast<uint16_t>(h23 >> 16)};
+        if (!C::OUT_T) {
+          // Row grow, columns gcol .. gcol + 3.
+          if (grow >= p.out_rows) continue;
+          if (vec_ok && gcol + 4 <= p.out_cols) {
+            *reinterpret_cast<uint2 *>(p.out + grow * p.out_ld + gcol) = make_uint2(h01, h23);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (gcol + e < p.out_cols) p.out[grow * p.out_ld + gcol + e] = h[e];
+          }
+        } else {
+          // Column gcol of the tile = row gcol of the transposed output, its
+          // entries grow .. grow + 3.
+          if (gcol >= p.out_cols) continue;
+          if (vec_ok && grow + 4 <= p.out_rows) {
+            *reinterpret_cast<uint2 *>(p.out + gcol * p.out_ld + grow) = make_uint2(h01, h23);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (grow + e < p.out_rows) p.out[gcol * p.out_ld + grow + e] = h[e];
+          }
+        }
       }
     }
     cluster_sync_all();
