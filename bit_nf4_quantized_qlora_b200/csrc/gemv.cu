@@ -7,11 +7,13 @@
 // discard), so the kernel is a streaming pipeline whose decode costs about one
 // byte permute and one shared-memory load per two weights:
 //
-//   * one producer warp streams 16 KB tiles of packed codes (128 weight rows x
-//     4 NF4 blocks, 128-byte swizzled) into a shared-memory ring with TMA;
-//   * a 64 KB shared table maps every code byte (two weights) to the bf16 pair
-//     {NF4[hi nibble], NF4[lo nibble]}, with 32 lane-private copies 256 bytes
-//     apart so 32 lookups always hit 32 banks;
+//   * one producer warp streams each stage into a shared-memory ring with TMA:
+//     a 16 KB tile of packed codes (128 weight rows x 4 NF4 blocks) and the
+//     matching 16-token x 4-block slice of X, both 128-byte swizzled, on one
+//     mbarrier, so the consumers never wait on a global load of X;
+//   * a 32 KB shared table maps every code byte (two weights) to the bf16 pair
+//     {NF4[hi nibble], NF4[lo nibble]}, with 32 lane-private copies in each
+//     128-byte row so 32 lookups always hit 32 banks;
 //   * eight consumer warps (16 rows each) feed the pairs as the A operand of
 //     m16n8k16 tensor-core MMAs with X as the B operand; the four MMAs of an
 //     NF4 block accumulate into a fresh tile that is scaled by the block's
@@ -34,13 +36,18 @@ constexpr int kThreads = 32 * (kConsumers + 1);       // + one producer warp
 constexpr int kRows = 16 * kConsumers;                 // 128 weight rows per CTA
 constexpr int kStageBlocks = 4;                        // NF4 blocks of K per stage
 constexpr uint32_t kStageBytes = kRows * kStageBlocks * 32u;   // 16 KB
-constexpr int kStages = 2;                             // x 2 CTAs per SM
+constexpr int kStages = 3;                             // x 2 CTAs per SM
 constexpr int kMaxM = 16;
-constexpr uint32_t kLutBytes = kPairLutBytes;
-constexpr uint32_t kSmemBytes = kLutBytes + 1024u + kStages * kStageBytes + kMaxM * kRows * 4u;
+constexpr uint32_t kXBlockBytes = 16u * 128u;          // X slice of one NF4 block: 16 tokens x 64 bf16
+constexpr uint32_t kSlotBytes = kStageBytes + kStageBlocks * kXBlockBytes;   // codes tile, then X
+constexpr uint32_t kLutBytes = 256u * 128u;            // one 128-byte row per code byte
+constexpr uint32_t kRedBytes = kMaxM * kRows * 4u;     // partial sums, aliased onto the ring
+static_assert(kRedBytes <= kStages * kSlotBytes, "partial sums fit in the ring");
+constexpr uint32_t kSmemBytes = kLutBytes + 1024u + kStages * kSlotBytes;
 
 struct __align__(64) GemvParams {
   CUtensorMap tmCodes;          // codes as [n rows x k/2 bytes], box {128, 128}, 128B swizzle
+  CUtensorMap tmX;              // X as [m rows x k] bf16, box {64, 8 or 16}, 128B swizzle
   const uint16_t *X;
   const uint8_t *absmax_q;
   const float *group_scale;
@@ -51,9 +58,32 @@ struct __align__(64) GemvParams {
   unsigned *err;
   int64_t n, k;
   int m, r;
+  uint32_t x_box_bytes;         // bytes of one X box (64 columns x 8 or 16 token rows)
   Nf4Tables tab;
 };
 
+// The byte-pair table: row b (128 bytes) holds 32 copies of the bf16 pair
+// {NF4[b >> 4], NF4[b & 15]}, one per lane.
+__device__ __forceinline__ void build_lut(uint8_t *lut, const Nf4Tables &tab, int tid, int nthreads) {
+  uint4 *lw = reinterpret_cast<uint4 *>(lut);
+  for (int i = tid; i < 256 * 8; i += nthreads) {
+    const int b = i >> 3;
+    const uint32_t v = pack_bf16x2(tab.level[b >> 4], tab.level[b & 15]);
+    lw[i] = make_uint4(v, v, v, v);
+  }
+}
+// Table offset of byte J (0..3) of `word` for the lane whose lane*4 is lane4.
+template <int J>
+__device__ __forceinline__ uint32_t lut_off(uint32_t word, uint32_t lane4) {
+  const uint32_t sh = J == 0 ? (word << 7) : (word >> (8 * J - 7));
+  return (sh & 0x7F80u) | lane4;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
@@ -79,15 +109,15 @@ __device__ __forceinline__ void block_mma(float (&bacc)[TOK_TILES][4], uint2 c0,
     const uint32_t w1 = ss < 2 ? c1.x : c1.y;
     uint32_t a[4];
     if ((ss & 1) == 0) {
-      a[0] = *reinterpret_cast<const uint32_t *>(lut + pair_lut_off<0>(w0, lane4));
-      a[1] = *reinterpret_cast<const uint32_t *>(lut + pair_lut_off<0>(w1, lane4));
-      a[2] = *reinterpret_cast<const uint32_t *>(lut + pair_lut_off<1>(w0, lane4));
-      a[3] = *reinterpret_cast<const uint32_t *>(lut + pair_lut_off<1>(w1, lane4));
+      a[0] = *reinterpret_cast<const uint32_t *>(lut + lut_off<0>(w0, lane4));
+      a[1] = *reinterpret_cast<const uint32_t *>(lut + lut_off<0>(w1, lane4));
+      a[2] = *reinterpret_cast<const uint32_t *>(lut + lut_off<1>(w0, lane4));
+      a[3] = *reinterpret_cast<const uint32_t *>(lut + lut_off<1>(w1, lane4));
     } else {
-      a[0] = *reinterpret_cast<const uint32_t *>(lut + pair_lut_off<2>(w0, lane4));
-      a[1] = *reinterpret_cast<const uint32_t *>(lut + pair_lut_off<2>(w1, lane4));
-      a[2] = *reinterpret_cast<const uint32_t *>(lut + pair_lut_off<3>(w0, lane4));
-      a[3] = *reinterpret_cast<const uint32_t *>(lut + pair_lut_off<3>(w1, lane4));
+      a[0] = *reinterpret_cast<const uint32_t *>(lut + lut_off<2>(w0, lane4));
+      a[1] = *reinterpret_cast<const uint32_t *>(lut + lut_off<2>(w1, lane4));
+      a[2] = *reinterpret_cast<const uint32_t *>(lut + lut_off<3>(w0, lane4));
+      a[3] = *reinterpret_cast<const uint32_t *>(lut + lut_off<3>(w1, lane4));
     }
 #pragma unroll
     for (int t = 0; t < TOK_TILES; ++t) {
@@ -107,7 +137,8 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
   // link-time constant address); the TMA ring is 1024-aligned after it.
   const uint8_t *lut = dsmem;
   const uint32_t ring = (smem_u32(dsmem) + kLutBytes + 1023u) & ~1023u;
-  const uint32_t red_addr = ring + kStages * kStageBytes;
+  // The partial sums reuse the ring once every stage has been consumed.
+  const uint32_t red_addr = ring;
   float *red = reinterpret_cast<float *>(dsmem + (red_addr - smem_u32(dsmem)));
 
   const uint32_t crank = cluster_rank();
@@ -122,6 +153,11 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
   const int st_hi = static_cast<int>((static_cast<int64_t>(nst_all) * (crank + 1)) / csize);
   const int nst = st_hi - st_lo;
   const int kb_lo = st_lo * kStageBlocks;
+  // CTAs walk their stages from different starting points (rotated by the
+  // row tile's index), so that at any moment the CTAs read different slices
+  // of X rather than all hitting the same few L2 lines.
+  const int rot = nst > 0 ? static_cast<int>(blockIdx.x % static_cast<unsigned>(nst)) : 0;
+  const auto phys = [&](int st) { return st + rot < nst ? st + rot : st + rot - nst; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -130,8 +166,14 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
     }
     fence_mbar_init();
   }
-  build_pair_lut(dsmem, p.tab, threadIdx.x, kThreads);
+  build_lut(dsmem, p.tab, threadIdx.x, kThreads);
   __syncthreads();
+
+  const int g = lane >> 2, q = lane & 3;
+  const int lr0 = warp * 16 + g, lr1 = lr0 + 8;          // rows of the tile (rows past n are
+  float acc[TOK_TILES][4];                                // computed but never stored)
+#pragma unroll
+  for (int t = 0; t < TOK_TILES; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
 
   if (warp == kConsumers) {
     // ------------------------------------------------------------ producer
@@ -141,9 +183,13 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
         const int s = st % kStages;
         const uint32_t ph = static_cast<uint32_t>(st / kStages) & 1u;
         if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, p.err, kErrTimeoutEmpty)) break;
-        mbar_arrive_expect_tx(&full_bar[s], kStageBytes);
-        tma_load_2d(ring + s * kStageBytes, &p.tmCodes, &full_bar[s], (kb_lo + st * kStageBlocks) * 32,
-                    static_cast<int>(n_cta));
+        const int kb_st = kb_lo + phys(st) * kStageBlocks;
+        const int nb = kblocks - kb_st < kStageBlocks ? kblocks - kb_st : kStageBlocks;   // blocks of X inside K
+        mbar_arrive_expect_tx(&full_bar[s], kStageBytes + static_cast<uint32_t>(nb) * p.x_box_bytes);
+        const uint32_t slot = ring + s * kSlotBytes;
+        tma_load_2d(slot, &p.tmCodes, &full_bar[s], kb_st * 32, static_cast<int>(n_cta));
+        for (int b = 0; b < nb; ++b)
+          tma_load_2d(slot + kStageBytes + b * kXBlockBytes, &p.tmX, &full_bar[s], (kb_st + b) * 64, 0);
         ++issued;
       }
       for (int st = issued - kStages < 0 ? 0 : issued - kStages; st < issued; ++st)
@@ -152,8 +198,6 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
     }
   } else {
     // ------------------------------------------------------------ consumers
-    const int g = lane >> 2, q = lane & 3;
-    const int lr0 = warp * 16 + g, lr1 = lr0 + 8;          // rows of the tile (rows past n are
     const int64_t gr0 = n_cta + lr0 < p.n ? n_cta + lr0 : p.n - 1;   // computed but never stored)
     const int64_t gr1 = n_cta + lr1 < p.n ? n_cta + lr1 : p.n - 1;
     const int64_t b0 = gr0 * kblocks, b1 = gr1 * kblocks;
@@ -178,32 +222,44 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
     float t0 = 0.f, t1 = 0.f;
     int next0 = kb_lo, next1 = kb_lo;
 
-    float acc[TOK_TILES][4];
-#pragma unroll
-    for (int t = 0; t < TOK_TILES; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-
-    const uint4 *xp[TOK_TILES];
-    bool xok[TOK_TILES];
+    // Swizzled offsets of this lane's two 16-byte pieces of X (columns 16q ..
+    // 16q + 15 of token g + 8t) inside a block's X slice.
+    uint32_t xoff[TOK_TILES][2];
 #pragma unroll
     for (int t = 0; t < TOK_TILES; ++t) {
-      const int tok = g + 8 * t;
-      xok[t] = tok < p.m;
-      xp[t] = reinterpret_cast<const uint4 *>(p.X + static_cast<int64_t>(xok[t] ? tok : 0) * p.k +
-                                              static_cast<int64_t>(kb_lo) * 64 + 16 * q);
+      const uint32_t row = static_cast<uint32_t>(g + 8 * t) * 128u;
+      xoff[t][0] = row + ((static_cast<uint32_t>(2 * q) ^ static_cast<uint32_t>(g)) << 4);
+      xoff[t][1] = row + ((static_cast<uint32_t>(2 * q + 1) ^ static_cast<uint32_t>(g)) << 4);
     }
 
     bool ok = true;
+    // Absmax code words of a whole stage (4-aligned blocks, stage inside K),
+    // loaded one stage ahead so that their latency hides under a stage.
+    const auto stage_words = [&](int st_, uint32_t &w0, uint32_t &w1) {
+      const int sp_ = phys(st_);
+      if (qwords && kb_lo + (sp_ + 1) * kStageBlocks <= kblocks) {
+        w0 = __ldg(reinterpret_cast<const uint32_t *>(q0p + sp_ * kStageBlocks));
+        w1 = __ldg(reinterpret_cast<const uint32_t *>(q1p + sp_ * kStageBlocks));
+      }
+    };
+    uint32_t wn0 = 0, wn1 = 0;
+    if (nst > 0) stage_words(0, wn0, wn1);
     for (int st = 0; st < nst && ok; ++st) {
       const int s = st % kStages;
       const uint32_t ph = static_cast<uint32_t>(st / kStages) & 1u;
-      const int kb_st = kb_lo + st * kStageBlocks;
+      const uint32_t wc0 = wn0, wc1 = wn1;
+      if (st + 1 < nst) stage_words(st + 1, wn0, wn1);
+      const int sp = phys(st);
+      const int kb_st = kb_lo + sp * kStageBlocks;
+      // Back at the start of the CTA's K range: the group constants are
+      // looked up afresh.
+      if (sp == 0 && st > 0) next0 = next1 = kb_lo;
       const bool full = kb_st + kStageBlocks <= kblocks;
-      // Absmax codes and X of this stage, issued before the wait.
+      // Absmax codes of this stage (prefetched on the word path).
       float qf0[kStageBlocks], qf1[kStageBlocks];
       bool qv[kStageBlocks];
       if (full && qwords) {
-        const uint32_t w0 = __ldg(reinterpret_cast<const uint32_t *>(q0p + st * kStageBlocks));
-        const uint32_t w1 = __ldg(reinterpret_cast<const uint32_t *>(q1p + st * kStageBlocks));
+        const uint32_t w0 = wc0, w1 = wc1;
         if (fp8) {
 #pragma unroll
           for (int b = 0; b < kStageBlocks; ++b) {
@@ -220,21 +276,8 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
 #pragma unroll
         for (int b = 0; b < kStageBlocks; ++b) {
           qv[b] = kb_st + b < kblocks;
-          qf0[b] = qv[b] ? code_value(__ldg(q0p + st * kStageBlocks + b), fp8) : 0.f;
-          qf1[b] = qv[b] ? code_value(__ldg(q1p + st * kStageBlocks + b), fp8) : 0.f;
-        }
-      }
-      uint4 xa[kStageBlocks][TOK_TILES], xb[kStageBlocks][TOK_TILES];
-#pragma unroll
-      for (int b = 0; b < kStageBlocks; ++b) {
-#pragma unroll
-        for (int t = 0; t < TOK_TILES; ++t) {
-          xa[b][t] = make_uint4(0u, 0u, 0u, 0u);
-          xb[b][t] = make_uint4(0u, 0u, 0u, 0u);
-          if (xok[t] && (full || kb_st + b < kblocks)) {
-            xa[b][t] = __ldg(xp[t] + (st * kStageBlocks + b) * 8);
-            xb[b][t] = __ldg(xp[t] + (st * kStageBlocks + b) * 8 + 1);
-          }
+          qf0[b] = qv[b] ? code_value(__ldg(q0p + sp * kStageBlocks + b), fp8) : 0.f;
+          qf1[b] = qv[b] ? code_value(__ldg(q1p + sp * kStageBlocks + b), fp8) : 0.f;
         }
       }
       // Group constants: with 4-aligned blocks a group boundary falls on a
@@ -247,16 +290,29 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
         t1 = group_constant(__ldg(p.group_scale + ((b1 + kb_st) >> 8)), fp8);
         next1 = kb_st + 256 - static_cast<int>((b1 + kb_st) & 255);
       }
-      ok = mbar_wait_bounded(&full_bar[s], ph, p.err, kErrTimeoutFullA);
+      // A wait that gives up (it never should) ends the warp's loop on every
+      // lane together, so the warp-collective MMAs below always see 32 lanes.
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full_bar[s], ph, p.err, kErrTimeoutFullA));
       if (!ok) break;
-      const uint32_t tile = ring + s * kStageBytes;
+      const uint32_t tile = ring + s * kSlotBytes;
+      const uint32_t xtile = tile + kStageBytes;
+      // A whole stage inside K and inside one group per row needs no
+      // per-block checks (the checks are scalar; every lane runs the same
+      // MMAs either way).
       const bool fast = full && next0 >= kb_st + kStageBlocks && next1 >= kb_st + kStageBlocks;
 #pragma unroll
       for (int b = 0; b < kStageBlocks; ++b) {
         const uint2 c0 = lds64(tile + off0[b]);
         const uint2 c1 = lds64(tile + off1[b]);
+        // X of the block (zero past K, where its slice was not loaded).
+        uint4 xa[TOK_TILES], xb[TOK_TILES];
+#pragma unroll
+        for (int t = 0; t < TOK_TILES; ++t) {
+          xa[t] = qv[b] ? lds128(xtile + b * kXBlockBytes + xoff[t][0]) : make_uint4(0u, 0u, 0u, 0u);
+          xb[t] = qv[b] ? lds128(xtile + b * kXBlockBytes + xoff[t][1]) : make_uint4(0u, 0u, 0u, 0u);
+        }
         float bacc[TOK_TILES][4];
-        block_mma<TOK_TILES>(bacc, c0, c1, xa[b], xb[b], lut, lane4);
+        block_mma<TOK_TILES>(bacc, c0, c1, xa, xb, lut, lane4);
         if (!fast) {
           const int kb = kb_st + b;
           if (kb == next0 && kb < kblocks) {
@@ -282,6 +338,11 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_fwd_kernel(const __grid_cons
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[s]);
     }
+  }
+  // Every stage is consumed and every copy has landed (the producer drained
+  // its ring): the partial sums may now overwrite it.
+  __syncthreads();
+  if (warp < kConsumers) {
     // Partial sums: rows lr0/lr1, tokens 2q, 2q+1 (+8t); red is [token][row].
 #pragma unroll
     for (int t = 0; t < TOK_TILES; ++t) {
@@ -406,6 +467,11 @@ cudaError_t launch_gemv_fwd(const uint16_t *X, int64_t m, const uint8_t *codes, 
   if (m <= 0) return cudaSuccess;
   GemvParams p{};
   if (!encode_codes_map(&p.tmCodes, codes, n, k / 2, 128, kRows, true)) return cudaErrorInvalidValue;
+  // X boxes of 64 columns and 8 (m <= 8) or 16 token rows; rows past m read
+  // as zero.
+  const uint32_t x_rows = m <= 8 ? 8u : 16u;
+  if (!encode_bf16_map(&p.tmX, X, m, k, 64, x_rows)) return cudaErrorInvalidValue;
+  p.x_box_bytes = 128u * x_rows;
   p.X = X;
   p.absmax_q = absmax_q;
   p.group_scale = group_scale;
@@ -433,22 +499,15 @@ cudaError_t launch_gemv_fwd(const uint16_t *X, int64_t m, const uint8_t *codes, 
                                      configured2);
     if (e != cudaSuccess) return e;
   }
-  // Split K over a cluster of cs CTAs.  Pick cs in 1..8 to fill the resident
-  // CTA slots (two per SM) in as few, as full waves as possible, keeping at
-  // least two stages of K per CTA.
+  // Split K over a cluster of cs CTAs: the smallest cs in 1..8 that puts a
+  // CTA on every SM, keeping at least two stages of K per CTA.  Each CTA
+  // pays for its table, its ring fill and a cluster reduction, so splitting
+  // further (to fill both CTA slots of every SM, or whole waves) costs more
+  // than the idle slots do.
   const int64_t row_ctas = (n + kRows - 1) / kRows;
   const int64_t kblocks = k / 64;
-  const int64_t slots = 2LL * sms;
   int cs = 1;
-  double best = -1.0;
-  for (int c = 1; c <= 8; ++c) {
-    if (c > 1 && (kblocks / kStageBlocks) / c < 2) break;
-    const int64_t ctas = row_ctas * c;
-    const int64_t waves = (ctas + slots - 1) / slots;
-    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
-    // Fuller waves first; among equal, fewer CTAs (less reduction traffic).
-    if (eff > best + 1e-9) { best = eff; cs = c; }
-  }
+  while (cs < 8 && row_ctas * cs < sms && (kblocks / kStageBlocks) / (cs + 1) >= 2) ++cs;
 
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(row_ctas), static_cast<unsigned>(cs), 1);

@@ -45,6 +45,19 @@
 namespace qlora {
 namespace {
 
+// 16 bytes (four fp32) at the same offset in CTA `rank`'s shared memory;
+// local_addr must be 16-byte aligned.
+__device__ __forceinline__ float4 ld_dsmem_v4(uint32_t local_addr, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(remote)
+               : "memory");
+  return v;
+}
+
 constexpr int kBK = 64;                       // k-step: 64 bf16 = one swizzle row
 constexpr uint32_t kASub = 128u * kBK * 2u;   // 16 KB: one 128-row A tile
 
