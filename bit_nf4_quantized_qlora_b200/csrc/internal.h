@@ -76,6 +76,10 @@ bool encode_bf16_map(CUtensorMap *m, const uint16_t *ptr, int64_t rows, int64_t 
 // slab's rows and columns.
 bool encode_f32_slab_map(CUtensorMap *m, const float *ptr, int64_t slabs, int64_t rows, int64_t cols,
                          uint32_t box_cols, uint32_t box_rows);
+// fp32 row-major [rows x cols], box {box_cols, box_rows}, 128-byte swizzle
+// (box_cols * 4 <= 128).
+bool encode_f32_map(CUtensorMap *m, const float *ptr, int64_t rows, int64_t cols, uint32_t box_cols,
+                    uint32_t box_rows);
 bool encode_codes_map(CUtensorMap *m, const uint8_t *ptr, int64_t rows, int64_t row_bytes, uint32_t box_bytes,
                       uint32_t box_rows, bool swizzle128);
 

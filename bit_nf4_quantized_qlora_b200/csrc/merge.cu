@@ -6,308 +6,244 @@
 // one fused multiply-add, W^ + s * acc, acc the fp32 sum of the rank-r
 // product, and rounded once to bf16 for the bf16 export.
 //
-// The output is cut into tiles of 128 rows x 128 columns (8 warps of 32 x 64
-// per tile), and every CTA that fits on the GPU at once takes an equal run of
-// them in band-major order, so a run crosses into a new band of 128 rows at
-// most once or twice.  The band's 128 rows of B stay in shared memory; each
-// tile's r x 128 slice of A (rows padded to 272 bytes), its code bytes and its
-// 256 block constants c' go through a double buffer filled by asynchronous
-// 16-byte copies one tile ahead, so the copies of the next tile run under the
-// current tile's MMAs and epilogue.  Each warp accumulates B . A on m16n8k16
-// tensor-core MMAs (A operand = rows of B as 32-bit words, B operand =
-// columns of A by ldmatrix.trans, two n8 tiles per load, shared by the warp's
-// two m16 tiles).  Each row of a warp's piece is one NF4 block, so the
-// epilogue decodes it through one per-row bf16 table of the block's 16
-// scaled levels (byte permutes, no per-element lookups), adds s . acc in
-// fp32, and writes 16 rows at a time through a shared-memory stage as
-// 16-byte row segments.  The floor is HBM on the output writes (2 or 4 bytes
-// per weight against 0.52 read); what bounds it is instruction issue.
+// One CTA per output tile of 128 rows x 256 columns.  One thread stages the
+// tile's operands by TMA, 128-byte swizzled: the tile's 128 rows of B (K-major,
+// 64 ranks per slab; ranks past r read as zero), the 64 x 256 slice of A
+// (MN-major, four 64-column slabs) and the tile's packed codes (128 rows x
+// 128 bytes); it issues the tcgen05 MMAs of B . A into a 128 x 256 fp32
+// accumulator in tensor memory (r > 64 walks 64-rank slabs through the same
+// buffers).  Eight epilogue warps then each own 32 accumulator rows (the
+// tensor-memory lane quarter of their warp) and one half of the columns:
+// a thread reads its row's accumulator 32 columns at a time with
+// tcgen05.ld, decodes the row's NF4 block through one bf16 table of the
+// block's 16 scaled levels (byte permutes, no per-element lookups), forms
+// W' = fma(s, acc, W^) in fp32 and writes the row into a 128-byte-swizzled
+// staging tile, which one thread of the half stores with TMA.  The floor is
+// HBM on the output writes (2 or 4 bytes per weight against 0.52 read).
 #include "common.cuh"
 #include "internal.h"
+#include "tcgen05.cuh"
 
 namespace qlora {
 namespace {
 
-constexpr int kTM = 128, kTN = 128;
-constexpr int kWarps = 8, kThreads = 32 * kWarps;
+constexpr int kTM = 128, kTN = 256;               // tile rows x columns
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;     // warp 0: TMA + MMA, warp 1: tensor memory, 2..9: epilogue
 constexpr int kMaxR = 256;
+constexpr uint32_t kBSlab = kTM * 128u;           // 16 KB: 128 rows of B x 64 ranks
+constexpr uint32_t kASlab = 4u * 8192u;           // 32 KB: 64 ranks x 256 columns of A (four 64-column slabs)
+constexpr uint32_t kCodeTile = kTM * 128u;        // 16 KB: 128 rows x 4 blocks of codes
+constexpr uint32_t kStage = kTM * 128u;           // 16 KB: one staged box per half of the epilogue
+constexpr uint32_t kOffB = 0, kOffA = kBSlab, kOffCodes = kOffA + kASlab, kOffStage = kOffCodes + kCodeTile;
+constexpr uint32_t kTmemCols = kTN;
+constexpr uint32_t kIdesc = make_idesc(kTN, false, true);
 
-struct MergeParams {
-  const uint8_t *codes;
+struct __align__(64) MergeParams {
+  CUtensorMap tmB;        // B [n x r] bf16, box {64, 128}
+  CUtensorMap tmA;        // A [r x k] bf16, box {64, 64}
+  CUtensorMap tmCodes;    // codes [n x k/2] bytes, box {128, 128}
+  CUtensorMap tmOutH;     // W' bf16 [n x k], box {64, 128}
+  CUtensorMap tmOutF;     // W' fp32 [n x k], box {32, 128}
   const uint8_t *absmax_q;
   const float *group_scale;
-  const float *mu;          // E4M3 + mean absmax format: the tensor mean; else null
-  const uint16_t *A;      // [r x k]
-  const uint16_t *B;      // [n x r]
-  uint16_t *out_bf16;     // [n x k] or null
-  float *out_f32;         // [n x k] or null
+  const float *mu;        // E4M3 + mean absmax format: the tensor mean; else null
+  unsigned *err;
   int64_t n, k;
   int r;
-  int nbuf;               // tile buffers in shared memory (2: copies one tile ahead)
+  int out_h, out_f;       // which exports are written
   float scale;
   Nf4Tables tab;
 };
 
-// Shared-memory layout (bytes), for rank r.  Padding puts the 32 lanes of
-// each access pattern in 32 distinct banks:
-//   rows of B, r/2 + 4 words: fragment reads (rows g, words q) hit 4g + q;
-//   rows of the A slice, 256 + 16 bytes: the eight 16-byte rows of an
-//     ldmatrix piece start four banks apart;
-//   rows of code bytes, 80 bytes: rows g start at banks 20g mod 32;
-//   stage rows, 36 words (bf16 pairs) or 72 words (fp32): stores of rows g
-//     hit 4g + 4t + q, or 8g + 8t + 2q per half-warp.
-constexpr uint32_t kARowBytes = kTN * 2u + 16u;
-constexpr uint32_t kCodeRow = 80u;
-constexpr int kStageH = 36, kStageF = 72;                 // words per stage row
-constexpr uint32_t kStageWarpBytes = 16u * kStageF * 4u;  // 16 rows, the larger of the two
-constexpr uint32_t kSmemCap = 227u * 1024u;
-struct Layout {
-  uint32_t row_words, bs, buf, at, codes, cp, buf_bytes, stage, total;
-  __host__ __device__ Layout(int r, int nbuf) {
-    row_words = static_cast<uint32_t>(r / 2 + 4);
-    bs = 0;
-    // Per-tile buffer (two of them): A slice, code bytes, block constants.
-    buf = (bs + kTM * row_words * 4u + 15u) & ~15u;
-    at = 0;
-    codes = at + static_cast<uint32_t>(r) * kARowBytes;
-    cp = codes + kTM * kCodeRow;
-    buf_bytes = (cp + kTM * 2 * 4u + 15u) & ~15u;
-    stage = buf + static_cast<uint32_t>(nbuf) * buf_bytes;
-    total = stage + kWarps * kStageWarpBytes;
-  }
-};
-
-// 16-byte global -> shared copy that bypasses registers (zeros when !valid;
-// src is then a valid address that is not read).
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
-               : "memory");
+// AND of v over the `count` threads that take barrier `id` (a multiple of 32).
+__device__ __forceinline__ bool barrier_and(uint32_t id, uint32_t count, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
 }
 
-template <bool F32>
 __global__ void __launch_bounds__(kThreads, 2) merge_kernel(const __grid_constant__ MergeParams p) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  const Layout L(p.r, p.nbuf);
-  uint32_t *bs = reinterpret_cast<uint32_t *>(sm + L.bs);
-  const uint32_t sbase = smem_u32(sm);
+  extern __shared__ uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t codes_bar;   // the codes tile landed (one phase)
+  __shared__ __align__(8) uint64_t full_bar;    // a slab of B and A landed (one phase per slab)
+  __shared__ __align__(8) uint64_t mma_bar;     // a slab's MMAs finished reading (one phase per slab but the last)
+  __shared__ __align__(8) uint64_t acc_bar;     // the accumulator is complete (one phase)
+  __shared__ uint32_t tmem_slot;
 
-  // This CTA's run of tiles in band-major order: [t_begin, t_end) of
-  // bands x tiles_k, split evenly over the grid.
-  const int tiles_k = static_cast<int>((p.k + kTN - 1) / kTN);
-  const int64_t bands = (p.n + kTM - 1) / kTM;
-  const int64_t total = bands * tiles_k;
-  const int64_t t_begin = total * blockIdx.x / gridDim.x;
-  const int64_t t_end = total * (blockIdx.x + 1) / gridDim.x;
-  const int tid = threadIdx.x;
-  const int rw = static_cast<int>(L.row_words);
-  const int chunks_r = p.r / 8;   // 16-byte pieces of a row of B
+  const uint32_t base = (smem_u32(dsmem) + 1023u) & ~1023u;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kTM;   // first row of the tile
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kTN;   // first column
+  const int nslabs = (p.r + 63) / 64;
 
-  // The band's 128 rows of B (a padded row is 2r + 16 bytes, a multiple of
-  // 16); zeros past n.
-  const auto issue_band = [&](int64_t n0) {
-    for (int i = tid; i < kTM * chunks_r; i += kThreads) {
-      const int row = i / chunks_r, c = i % chunks_r;
-      const bool ok = n0 + row < p.n;
-      cp_async16(sbase + L.bs + static_cast<uint32_t>(row * rw + 4 * c) * 4u,
-                 ok ? static_cast<const void *>(p.B + (n0 + row) * p.r + 8 * c) : p.B, ok);
-    }
-  };
-  // One tile's r x 128 slice of A (row-major) and code bytes (128 rows x 64
-  // bytes) into buffer `b`; zeros past n and k.
-  const auto issue_tile = [&](int64_t n0, int ct, int b) {
-    const int64_t c0 = static_cast<int64_t>(ct) * kTN;
-    const uint32_t bb = sbase + L.buf + static_cast<uint32_t>(b) * L.buf_bytes;
-    for (int i = tid; i < p.r * (kTN / 8); i += kThreads) {
-      const int j = i / (kTN / 8), c = i % (kTN / 8);
-      const bool ok = c0 + 8 * c < p.k;
-      cp_async16(bb + L.at + static_cast<uint32_t>(j) * kARowBytes + 16u * c,
-                 ok ? static_cast<const void *>(p.A + static_cast<int64_t>(j) * p.k + c0 + 8 * c) : p.A, ok);
-    }
-    for (int i = tid; i < kTM * 4; i += kThreads) {
-      const int row = i >> 2, c = i & 3;
-      const bool ok = n0 + row < p.n && c0 + 32 * c < p.k;
-      cp_async16(bb + L.codes + static_cast<uint32_t>(row) * kCodeRow + 16u * c,
-                 ok ? static_cast<const void *>(p.codes + ((n0 + row) * p.k + c0) / 2 + 16 * c) : p.codes, ok);
-    }
-  };
-  const bool fp8 = p.mu != nullptr;
-  const float mu = load_mu(p.mu);
-  // W' = fma(s, acc, W^).  Without an adapter the sum starts at -0 and s is
-  // 1, which returns W^ exactly (-0 + x = x for every x, FP4's -0 level
-  // included), so no element needs a branch.
-  const float acc0 = p.r > 0 ? 0.f : -0.f;
-  const float s_eff = p.r > 0 ? p.scale : 1.f;
-  // c' of this thread's block of a tile (row tid / 2, block tid % 2).
-  const auto cprime = [&](int64_t n0, int ct) {
-    const int row = tid >> 1, b = tid & 1;
-    const int64_t c0 = static_cast<int64_t>(ct) * kTN;
-    float c = 0.f;
-    if (n0 + row < p.n && c0 + 64 * b < p.k) {
-      const int64_t blk = ((n0 + row) * p.k + c0) / 64 + b;
-      const float sg = __ldg(p.group_scale + (blk >> 8));
-      c = block_constant(__ldg(p.absmax_q + blk), fp8 ? sg : div255_rn(sg), fp8, mu);
-    }
-    return c;
-  };
-  float c_next = 0.f;
-  if (t_begin < t_end) {
-    const int64_t n0 = (t_begin / tiles_k) * kTM;
-    const int ct = static_cast<int>(t_begin % tiles_k);
-    issue_band(n0);
-    issue_tile(n0, ct, 0);
-    c_next = cprime(n0, ct);
+  if (threadIdx.x == 0) {
+    mbar_init(&codes_bar, 1);
+    mbar_init(&full_bar, 1);
+    mbar_init(&mma_bar, 1);
+    mbar_init(&acc_bar, 1);
+    fence_mbar_init();
   }
-  asm volatile("cp.async.commit_group;" ::: "memory");
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
 
-  // Copy groups: each tile's copies are one group, committed either at the
-  // top of the tile before it (a prefetch within the band, two buffers) or at
-  // the end of that tile (a new band, whose rows of B replace the old ones
-  // once every warp is done with them, or a single buffer).  Every top
-  // commits a group (possibly empty), so waiting for all but the newest
-  // group finds this tile's copies done.
-  for (int64_t tile = t_begin, it = 0; tile < t_end; ++tile, ++it) {
-    const int b = p.nbuf == 2 ? static_cast<int>(it & 1) : 0;
-    const int64_t band = tile / tiles_k;
-    const int64_t n0 = band * kTM;
-    const int ct = static_cast<int>(tile % tiles_k);
-    const bool has_next = tile + 1 < t_end;
-    const bool same_band = has_next && (tile + 1) / tiles_k == band;
-    const bool prefetch = p.nbuf == 2 && same_band;
-    uint8_t *cs = sm + L.buf + static_cast<uint32_t>(b) * L.buf_bytes + L.codes;
-    float *cp = reinterpret_cast<float *>(sm + L.buf + static_cast<uint32_t>(b) * L.buf_bytes + L.cp);
-    cp[tid] = c_next;
-    // The next tile's copies run under this tile's MMAs and epilogue.
-    if (prefetch) issue_tile(n0, ct + 1, b ^ 1);
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    if (prefetch) c_next = cprime(n0, ct + 1);
-    asm volatile("cp.async.wait_group 1;" ::: "memory");
-    __syncthreads();
-    const int64_t c0 = static_cast<int64_t>(ct) * kTN;
-    const uint32_t at_base = L.buf + static_cast<uint32_t>(b) * L.buf_bytes + L.at;
-
-    const int warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, q = lane & 3;
-    const int rg = warp & 3, ch = warp >> 2;   // rows 32 rg .. +32, columns 64 ch .. +64
-    float acc[2][8][4];
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&codes_bar, kCodeTile);
+      tma_load_2d(base + kOffCodes, &p.tmCodes, &codes_bar, static_cast<int>(c0 / 2), static_cast<int>(r0));
+      for (int j = 0; j < nslabs; ++j) {
+        // The buffers are free once the previous slab's MMAs have read them.
+        if (j > 0 && !mbar_wait_bounded(&mma_bar, static_cast<uint32_t>(j - 1) & 1u, p.err, kErrTimeoutEmpty)) break;
+        mbar_arrive_expect_tx(&full_bar, kBSlab + kASlab);
+        tma_load_2d(base + kOffB, &p.tmB, &full_bar, 64 * j, static_cast<int>(r0));
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int t = 0; t < 8; ++t) acc[mt][t][0] = acc[mt][t][1] = acc[mt][t][2] = acc[mt][t][3] = acc0;
-    const uint32_t *ar[2] = {bs + (32 * rg + g) * rw, bs + (32 * rg + 16 + g) * rw};
-    // ldmatrix.x4.trans for n8 tiles t, t + 1: lane l addresses row (l & 7) of
-    // piece l >> 3; pieces 0 / 1 are k rows 0..7 / 8..15 of tile t (its b0 /
-    // b1), pieces 2 / 3 the same of tile t + 1.
-    const uint32_t lm_row = static_cast<uint32_t>(((lane >> 3) & 1) * 8 + (lane & 7));
-    const uint32_t lm_col = static_cast<uint32_t>(64 * ch + (lane >> 4) * 8);
-    const uint32_t lm_base = smem_u32(sm) + at_base + lm_row * kARowBytes + 2u * lm_col;
-    for (int kk = 0; kk < p.r / 16; ++kk) {
-      uint32_t a[2][4];
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        a[mt][0] = ar[mt][8 * kk + q];
-        a[mt][1] = ar[mt][8 * rw + 8 * kk + q];
-        a[mt][2] = ar[mt][8 * kk + 4 + q];
-        a[mt][3] = ar[mt][8 * rw + 8 * kk + 4 + q];
-      }
-#pragma unroll
-      for (int t = 0; t < 8; t += 2) {
-        uint32_t b[4];
-        const uint32_t addr = lm_base + static_cast<uint32_t>(kk) * 16u * kARowBytes + 16u * static_cast<uint32_t>(t);
-        asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3])
-                     : "r"(addr));
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-          mma_bf16_16816(acc[mt][t], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b[0], b[1]);
-          mma_bf16_16816(acc[mt][t + 1], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b[2], b[3]);
+        for (int s = 0; s < 4; ++s)
+          tma_load_2d(base + kOffA + 8192u * s, &p.tmA, &full_bar, static_cast<int>(c0) + 64 * s, 64 * j);
+        if (!mbar_wait_bounded(&full_bar, static_cast<uint32_t>(j) & 1u, p.err, kErrTimeoutFullA)) {
+          // Let the copies in flight land before the CTA's memory is released.
+          mbar_wait_bounded(&full_bar, static_cast<uint32_t>(j) & 1u, p.err, kErrTimeoutDrain);
+          break;
         }
+        tc_fence_after();
+        const int ksteps = (p.r - 64 * j) / 16 < 4 ? (p.r - 64 * j) / 16 : 4;   // r is a multiple of 16
+        for (int kk = 0; kk < ksteps; ++kk) {
+          const uint64_t ad = smem_desc(base + kOffB + 32u * kk, 16u, 1024u);
+          const uint64_t bd = smem_desc(base + kOffA + 2048u * kk, 8192u, 1024u);
+          umma_f16(tmem, ad, bd, kIdesc, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(j + 1 < nslabs ? &mma_bar : &acc_bar);
       }
     }
-
-    // Epilogue.  Each row of the warp's 32 x 64 piece is one NF4 block, so a
-    // lane decodes its row's codes through one per-row bf16 table: lane (g, q)
-    // holds columns 8t + 2q, 8t + 2q + 1 of n8 tiles t = 0..7, whose shared
-    // code byte is byte q of word t of the row's 32 code bytes (high nibble
-    // first).  The lane gathers those eight bytes into two words and expands
-    // them into the eight bf16 pairs of W^ in tile order.
-    float *stage = reinterpret_cast<float *>(sm + L.stage + static_cast<uint32_t>(warp) * kStageWarpBytes);
-    uint32_t *stage_h = reinterpret_cast<uint32_t *>(stage);
-    const uint32_t sel_q = static_cast<uint32_t>(q) | (static_cast<uint32_t>(q + 4) << 4);
-    const int64_t gcol0 = c0 + 64 * ch;
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;
+    const int quad = warp & 3;                // tensor-memory lanes 32 quad .. 32 quad + 31
+    const int half = ew >> 2;                 // blocks 2 half and 2 half + 1 of the tile
+    const int row = quad * 32 + lane;         // tile row of this thread
+    const int64_t grow = r0 + row;
+    const bool leader = (ew & 3) == 0 && lane == 0;
+    const uint32_t bar_id = 1u + static_cast<uint32_t>(half);
+    const uint32_t stage_h = base + kOffStage + static_cast<uint32_t>(half) * kStage;
+    const uint32_t stage_f = base + kOffStage + (p.out_h ? 2u * kStage : 0u) + static_cast<uint32_t>(half) * kStage;
+    const uint32_t sw = static_cast<uint32_t>(row & 7);
+    const bool fp8 = p.mu != nullptr;
+    const float mu = load_mu(p.mu);
+    // W' = fma(s, acc, W^).  Without an adapter the sum is -0 and s is 1,
+    // which returns W^ exactly (-0 + x = x for every x, FP4's -0 level
+    // included).
+    const float s_eff = p.r > 0 ? p.scale : 1.f;
+    // c' of the thread's two blocks, requested before the waits.
+    float cp[2];
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int row = 32 * rg + 16 * mt + g + 8 * h;
-        const uint4 *crow = reinterpret_cast<const uint4 *>(cs + row * kCodeRow + 32 * ch);
-        const uint4 v0 = crow[0], v1 = crow[1];
-        const uint32_t wlo = prmt(prmt(v0.x, v0.y, sel_q), prmt(v0.z, v0.w, sel_q), 0x5410);
-        const uint32_t whi = prmt(prmt(v1.x, v1.y, sel_q), prmt(v1.z, v1.w, sel_q), 0x5410);
-        Bf16Table tb;
-        make_table(p.tab, cp[row * 2 + ch], tb);
-        uint32_t wv[8];
-        decode8(wlo, tb, wv);
-        decode8(whi, tb, wv + 4);
-        const int lr = g + 8 * h;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const float m0 = __fmaf_rn(s_eff, acc[mt][t][2 * h], bf16lo_to_f32(wv[t]));
-          const float m1 = __fmaf_rn(s_eff, acc[mt][t][2 * h + 1], bf16hi_to_f32(wv[t]));
-          if (F32)
-            *reinterpret_cast<float2 *>(stage + lr * kStageF + 8 * t + 2 * q) = make_float2(m0, m1);
-          else
-            stage_h[lr * kStageH + 4 * t + q] = pack_bf16x2(m0, m1);
-        }
+    for (int bb = 0; bb < 2; ++bb) {
+      const int64_t gcol = c0 + 64 * (2 * half + bb);
+      cp[bb] = 0.f;
+      if (grow < p.n && gcol < p.k) {
+        const int64_t blk = (grow * p.k + gcol) / 64;
+        const float sg = __ldg(p.group_scale + (blk >> 8));
+        cp[bb] = block_constant(__ldg(p.absmax_q + blk), fp8 ? sg : div255_rn(sg), fp8, mu);
       }
-      __syncwarp();
-      // 16 rows of 64 columns leave as 16-byte row segments.
-      const int64_t grow0 = n0 + 32 * rg + 16 * mt;
-      if (gcol0 < p.k) {
-        if (F32) {
-          // 16 rows x 256 bytes: lane l writes piece l & 15 of rows l / 16 + 2i.
-          const int lr0 = lane >> 4, pc = lane & 15;
-          float *dst = p.out_f32 + (grow0 + lr0) * p.k + gcol0 + 4 * pc;
-          uint16_t *dsth = p.out_bf16 ? p.out_bf16 + (grow0 + lr0) * p.k + gcol0 + 4 * pc : nullptr;
+    }
+    bool ok = mbar_wait_bounded(&codes_bar, 0u, p.err, kErrTimeoutFullB);
+    if (ok && p.r > 0) ok = mbar_wait_bounded(&acc_bar, 0u, p.err, kErrTimeoutAcc);
+    // Every epilogue thread takes the same path (the halves' barriers and the
+    // warp-collective tensor-memory loads below need all of them).
+    ok = barrier_and(3u, 32u * kEpiWarps, ok);
+    tc_fence_after();
+    // A staging buffer of this half is rewritten only after the stores that
+    // read it have finished reading, and stored once all 128 rows are in.
+    const auto stage_free = [&]() {
+      if (leader) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      named_barrier_sync(bar_id, 128);
+    };
+    const auto stage_store = [&](const CUtensorMap *map, uint32_t src, int64_t x) {
+      fence_proxy_async_smem();
+      named_barrier_sync(bar_id, 128);
+      if (leader) {
+        tma_store_2d(map, src, static_cast<int>(x), static_cast<int>(r0));
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      }
+    };
+    if (ok) {
+#pragma unroll 1
+      for (int bb = 0; bb < 2; ++bb) {
+        const int blk = 2 * half + bb;
+        Bf16Table tb;
+        make_table(p.tab, cp[bb], tb);
+        const uint32_t crow = base + kOffCodes + static_cast<uint32_t>(row) * 128u;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int lr = lr0 + 2 * i;
-            if (grow0 + lr < p.n) {
-              const float4 v = *reinterpret_cast<const float4 *>(stage + lr * kStageF + 4 * pc);
-              *reinterpret_cast<float4 *>(dst + 2 * i * p.k) = v;
-              if (dsth) {
-                uint2 hh;
-                hh.x = pack_bf16x2(v.x, v.y);
-                hh.y = pack_bf16x2(v.z, v.w);
-                *reinterpret_cast<uint2 *>(dsth + 2 * i * p.k) = hh;
-              }
+        for (int hh = 0; hh < 2; ++hh) {
+          // 32 columns: the accumulator, the codes (16 bytes) and W^.
+          uint32_t v[32];
+          if (p.r > 0) {
+            tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(64 * blk + 32 * hh), v);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0x80000000u;   // -0
+          }
+          const uint4 cw = lds128(crow + ((static_cast<uint32_t>(2 * blk + hh) ^ sw) << 4));
+          uint32_t wv[16];
+          decode8(cw.x, tb, wv + 0);
+          decode8(cw.y, tb, wv + 4);
+          decode8(cw.z, tb, wv + 8);
+          decode8(cw.w, tb, wv + 12);
+          float m[32];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            m[2 * i] = __fmaf_rn(s_eff, __uint_as_float(v[2 * i]), bf16lo_to_f32(wv[i]));
+            m[2 * i + 1] = __fmaf_rn(s_eff, __uint_as_float(v[2 * i + 1]), bf16hi_to_f32(wv[i]));
+          }
+          if (p.out_h) {
+            // The previous block's store must have read the buffer; the wait
+            // comes after this block's first 32 columns are computed, so it
+            // overlaps them.
+            if (hh == 0) stage_free();
+            // Row `row` of the [128 x 64] bf16 box: 16-byte chunks 4 hh .. 4 hh + 3.
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint32_t w4[4] = {pack_bf16x2(m[8 * c + 0], m[8 * c + 1]), pack_bf16x2(m[8 * c + 2], m[8 * c + 3]),
+                                      pack_bf16x2(m[8 * c + 4], m[8 * c + 5]), pack_bf16x2(m[8 * c + 6], m[8 * c + 7])};
+              sts128(stage_h + static_cast<uint32_t>(row) * 128u + ((static_cast<uint32_t>(4 * hh + c) ^ sw) << 4), w4);
             }
           }
-        } else {
-          // 16 rows x 128 bytes: lane l writes piece l & 7 of rows l / 8 + 4i.
-          const int lr0 = lane >> 3, pc = lane & 7;
-          uint16_t *dst = p.out_bf16 + (grow0 + lr0) * p.k + gcol0 + 8 * pc;
+          if (p.out_f) {
+            // Row `row` of the [128 x 32] fp32 box of these 32 columns.
+            stage_free();
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int lr = lr0 + 4 * i;
-            if (grow0 + lr < p.n)
-              *reinterpret_cast<uint4 *>(dst + 4 * i * p.k) =
-                  *reinterpret_cast<const uint4 *>(stage_h + lr * kStageH + 4 * pc);
+            for (int c = 0; c < 8; ++c) {
+              const uint32_t w4[4] = {__float_as_uint(m[4 * c + 0]), __float_as_uint(m[4 * c + 1]),
+                                      __float_as_uint(m[4 * c + 2]), __float_as_uint(m[4 * c + 3])};
+              sts128(stage_f + static_cast<uint32_t>(row) * 128u + ((static_cast<uint32_t>(c) ^ sw) << 4), w4);
+            }
+            stage_store(&p.tmOutF, stage_f, c0 + 64 * blk + 32 * hh);
           }
         }
+        if (p.out_h) stage_store(&p.tmOutH, stage_h, c0 + 64 * blk);
       }
-      __syncwarp();   // the stage is rewritten by the next m16 tile
     }
-    // Every warp is done with this tile's buffers (and the band's rows of B)
-    // before they are refilled.
-    __syncthreads();
-    if (has_next && !prefetch) {
-      const int64_t nn0 = ((tile + 1) / tiles_k) * kTM;
-      const int nct = static_cast<int>((tile + 1) % tiles_k);
-      if (!same_band) issue_band(nn0);
-      issue_tile(nn0, nct, p.nbuf == 2 ? b ^ 1 : 0);
-      asm volatile("cp.async.commit_group;" ::: "memory");
-      c_next = cprime(nn0, nct);
-    }
+    if (leader) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
   }
 }
 
@@ -316,44 +252,34 @@ __global__ void __launch_bounds__(kThreads, 2) merge_kernel(const __grid_constan
 cudaError_t launch_merge(const WeightView &w, const uint16_t *A, const uint16_t *B, int32_t r, float scale,
                          uint16_t *out_bf16, float *out_f32, cudaStream_t stream) {
   if (r < 0 || r > kMaxR || r % 16 != 0) return cudaErrorInvalidValue;
+  if (w.n <= 0 || w.k <= 0 || (out_bf16 == nullptr && out_f32 == nullptr)) return cudaSuccess;
   MergeParams p{};
-  p.codes = w.codes;
+  if (r > 0) {
+    if (!encode_bf16_map(&p.tmB, B, w.n, r, 64, kTM)) return cudaErrorInvalidValue;
+    if (!encode_bf16_map(&p.tmA, A, r, w.k, 64, 64)) return cudaErrorInvalidValue;
+  }
+  if (!encode_codes_map(&p.tmCodes, w.codes, w.n, w.k / 2, 128, kTM, true)) return cudaErrorInvalidValue;
+  if (out_bf16 && !encode_bf16_map(&p.tmOutH, out_bf16, w.n, w.k, 64, kTM)) return cudaErrorInvalidValue;
+  if (out_f32 && !encode_f32_map(&p.tmOutF, out_f32, w.n, w.k, 32, kTM)) return cudaErrorInvalidValue;
   p.absmax_q = w.absmax_q;
   p.group_scale = w.group_scale;
   p.mu = w.mu;
-  p.A = r > 0 ? A : nullptr;
-  p.B = r > 0 ? B : nullptr;
-  p.out_bf16 = out_bf16;
-  p.out_f32 = out_f32;
+  p.err = device_error_word();
   p.n = w.n;
   p.k = w.k;
   p.r = r;
+  p.out_h = out_bf16 ? 1 : 0;
+  p.out_f = out_f32 ? 1 : 0;
   p.scale = scale;
   p.tab = *w.tab;
-  p.nbuf = Layout(r, 2).total <= kSmemCap ? 2 : 1;
-  const uint32_t smem = Layout(r, p.nbuf).total;
-  int dev = 0, sms = 148;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // The limit is raised once per device to the most any rank uses, so
-  // concurrent calls with different ranks never lower it under one another.
+  const uint32_t smem = kOffStage + (out_bf16 ? 2u * kStage : 0u) + (out_f32 ? 2u * kStage : 0u) + 1024u;
+  // The limit is raised once per device to the most any call uses.
   static std::atomic<bool> configured[kMaxDevicesPerProcess] = {};
-  static std::atomic<bool> configured_f32[kMaxDevicesPerProcess] = {};
-  const void *fn = out_f32 ? reinterpret_cast<const void *>(merge_kernel<true>)
-                           : reinterpret_cast<const void *>(merge_kernel<false>);
-  e = set_smem_once(fn, static_cast<int>(kSmemCap), out_f32 ? configured_f32 : configured);
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(merge_kernel),
+                                static_cast<int>(kOffStage + 4u * kStage + 1024u), configured);
   if (e != cudaSuccess) return e;
-  // Every CTA that fits at once takes an equal run of the bands x column
-  // tiles, in band-major order.
-  const int64_t tiles = ((w.n + kTM - 1) / kTM) * ((w.k + kTN - 1) / kTN);
-  const int per_sm = smem <= kSmemCap / 2 ? 2 : 1;
-  const int64_t slots = static_cast<int64_t>(per_sm) * sms;
-  const dim3 grid(static_cast<unsigned>(tiles < slots ? tiles : slots), 1, 1);
-  if (out_f32)
-    merge_kernel<true><<<grid, kThreads, smem, stream>>>(p);
-  else
-    merge_kernel<false><<<grid, kThreads, smem, stream>>>(p);
+  const dim3 grid(static_cast<unsigned>((w.k + kTN - 1) / kTN), static_cast<unsigned>((w.n + kTM - 1) / kTM), 1);
+  merge_kernel<<<grid, kThreads, smem, stream>>>(p);
   count_launches(1);
   return cudaGetLastError();
 }

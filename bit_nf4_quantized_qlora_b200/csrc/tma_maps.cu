@@ -61,6 +61,12 @@ bool encode_bf16_map(CUtensorMap *m, const uint16_t *ptr, int64_t rows, int64_t 
                   static_cast<uint64_t>(cols) * 2u, box_cols, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+bool encode_f32_map(CUtensorMap *m, const float *ptr, int64_t rows, int64_t cols, uint32_t box_cols,
+                    uint32_t box_rows) {
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ptr, static_cast<uint64_t>(cols), static_cast<uint64_t>(rows),
+                  static_cast<uint64_t>(cols) * 4u, box_cols, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 bool encode_codes_map(CUtensorMap *m, const uint8_t *ptr, int64_t rows, int64_t row_bytes, uint32_t box_bytes,
                       uint32_t box_rows, bool swizzle128) {
   return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, ptr, static_cast<uint64_t>(row_bytes),
