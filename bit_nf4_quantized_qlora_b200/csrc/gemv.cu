@@ -4,8 +4,8 @@
 //
 // At decode-sized M the layer is bound by reading the packed weights from HBM
 // ("QLoRA and Quantized Training", The idea: dequantize each block, multiply,
-// discard), so the kernel is a streaming pipeline whose decode costs about one
-// byte permute and one shared-memory load per two weights:
+// discard), so the kernel is a streaming pipeline whose decode costs two
+// integer ops (the table address) and one shared-memory load per two weights:
 //
 //   * one producer warp streams each stage into a shared-memory ring with TMA:
 //     a 16 KB tile of packed codes (128 weight rows x 4 NF4 blocks) and the
@@ -18,8 +18,9 @@
 //     m16n8k16 tensor-core MMAs with X as the B operand; the four MMAs of an
 //     NF4 block accumulate into a fresh tile that is scaled by the block's
 //     reconstructed absmax c' = q * fp32(S/255) and added to the running sum;
-//   * a cluster of CTAs splits K; partial tiles are reduced through
-//     distributed shared memory and the adapter term T . B^T is added before
+//   * when the 128-row tiles alone leave SMs empty, a cluster of CTAs splits
+//     K; partial tiles are reduced through distributed shared memory (in the
+//     ring's memory, free by then) and the adapter term T . B^T is added before
 //     Y is written once in bf16.  T comes from the preceding projection
 //     kernel, which this kernel overlaps (programmatic dependent launch) and
 //     waits for only before its epilogue.

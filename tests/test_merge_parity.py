@@ -22,8 +22,11 @@ from oracle import merge, quant
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
+# Ragged row and column tiles (tiles are 128 x 256), every rank-slab count of
+# the tensor-core kernel (ranks 16..64: one slab; 128, 192, 256: two to four
+# slabs through the same operand buffers), the three codebooks.
 CASES = [(520, 576, 16, "nf4"), (1024, 1024, 64, "nf4"), (136, 448, 32, "fp4"), (64, 128, 256, "int4"),
-         (4104, 4096, 64, "nf4")]
+         (4104, 4096, 64, "nf4"), (300, 704, 128, "nf4"), (264, 320, 192, "fp4")]
 
 
 def _setup(n, k, r, name, seed=950):
