@@ -110,9 +110,9 @@ struct Cfg {
   // stages, so that two CTAs share an SM.
   static constexpr int STAGES = B_NF4 ? (STAGES_RAW > 6 ? 6 : STAGES_RAW) : (EPI == kEpiDropoutAdd ? 2 : 4);
   static constexpr uint32_t SMEM_BYTES = STAGE_BYTES * STAGES + 1024u;
-  // NF4 modes: groups of 8 dequant warps take k-steps in turn (two groups for
-  // the K-major forward tile, one for the MN-major input-gradient tile).
-  static constexpr int DQ_GROUPS = B_NF4 ? (B_MN ? 1 : 2) : 0;
+  // NF4 modes: two groups of 8 dequant warps take k-steps in turn (the
+  // expansion of a k-step is latency-bound; two groups keep two in flight).
+  static constexpr int DQ_GROUPS = B_NF4 ? 2 : 0;
   // The masked-add epilogue regenerates the dropout mask (one Philox call per
   // 16 outputs): sixteen warps share that work.
   static constexpr int NUM_EPI_WARPS = B_NF4 ? 8 * DQ_GROUPS : (EPI == kEpiDropoutAdd ? 16 : 4);
