@@ -936,9 +936,13 @@ def reference_step_sample(rows: int = 8, out_rows_frac: float = 1.0 / 64) -> dic
     from oracle import linear, quant
     items = _ref_prepare(rows, out_rows_frac)
     flops = 0
+    t_quant, n_quant = 0.0, 0
     t0 = time.perf_counter()
     for c, C, W, X, dY, A, Bm in items:
+        tq = time.perf_counter()
         packed, q, S, _ = quant.quantize_nf4_dq(W)
+        t_quant += time.perf_counter() - tq
+        n_quant += W.size
         W_hat = quant.dequant_bf16_values(packed, q, S).reshape(C, c.k)
         linear.fwd(X, W_hat, A, Bm, c.scale)
         linear.bwd_dx(dY, W_hat, A, Bm, c.scale)
@@ -949,7 +953,12 @@ def reference_step_sample(rows: int = 8, out_rows_frac: float = 1.0 / 64) -> dic
             "sample": f"per projection (gate, up, down): {rows} of the 4096 token rows x about "
                       f"{out_rows_frac:.4g} of the output rows -- oracle quantize + dequantize of those weight "
                       f"rows, fwd, bwd_dx and LoRA grads in fp64 (NumPy)",
-            "seconds": round(el, 3)}
+            "seconds": round(el, 3),
+            # NumPy's element-wise quantize runs on one thread (BLAS, in the
+            # linear algebra, uses `cores`).
+            "quantize": {"weights": int(n_quant), "seconds": round(t_quant, 3),
+                         "mweights_per_s": round(n_quant / t_quant / 1e6, 3) if t_quant > 0 else None,
+                         "threads": 1}}
 
 
 def run_reference(args):
