@@ -769,21 +769,25 @@ def run_ours(args):
     # End to end through the public API with host buffers.
     e2e = _e2e(projs, cases, flat, world, dev, stream, max(3, min(K, 10)))
 
-    m1 = _m1_decode(dev, peaks, peak_kind) if rank == 0 else None
-    decode_small = _decode_small_m(dev, peaks, peak_kind) if rank == 0 else None
+    # The per-GPU side measurements run in a single-GPU run only: with several
+    # ranks they would keep rank 0 busy for about a minute while the others
+    # wait in the closing barrier, and they say nothing about scaling.
+    single = world == 1
+    m1 = _m1_decode(dev, peaks, peak_kind) if single else None
+    decode_small = _decode_small_m(dev, peaks, peak_kind) if single else None
     # The standalone HBM-bound kernels run before the M-sweep and the decoder
     # block, after a short pause: right after seconds of dense GEMMs the same
     # calls measured up to 30 % slower for a second or two (clocks unchanged,
     # no throttle reason), which would misstate the kernels.
     qd = merged = codebook = None
-    if rank == 0:
+    if single:
         _settle(dev)
         qd = _quantize_dequant_70b(dev, peaks, peak_kind)
         merged = _merge_export(dev, peaks, peak_kind)
         codebook = _codebook_error(dev)
-    sweep = _up_proj_70b_sweep(dev, peaks, peak_kind) if rank == 0 else None
-    layer = _decoder_layer(dev) if rank == 0 else None
-    unfused = _unfused_comparator(projs[0], dev) if rank == 0 else None
+    sweep = _up_proj_70b_sweep(dev, peaks, peak_kind) if single else None
+    layer = _decoder_layer(dev) if single else None
+    unfused = _unfused_comparator(projs[0], dev) if single else None
     cpu = _cpu_baseline(rank, world)
 
     if rank == 0:
