@@ -26,8 +26,8 @@ WORKLOADS = {
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=("quantize", "dequant", "fwd", "fwd_nolora", "bwd_dx", "lora_bwd", "merge", "dropout",
-                                     "fwd_dropout", "bwd_dx_dropout"), required=True)
+    ap.add_argument("--op", choices=("quantize", "quantize_fp8", "dequant", "fwd", "fwd_nolora", "bwd_dx", "lora_bwd",
+                                     "merge", "dropout", "fwd_dropout", "bwd_dx_dropout"), required=True)
     ap.add_argument("--workload", choices=sorted(WORKLOADS), required=True)
     ap.add_argument("--m", type=int, default=4096)
     ap.add_argument("--iters", type=int, default=3)
@@ -39,7 +39,8 @@ def main(argv=None):
     case = WORKLOADS[a.workload](a.m)
     W = case.W().to(dev)
     w = B.qlora_quantize_nf4_dq(W)
-    if a.op != "quantize":
+    w8 = B.qlora_quantize_4bit_dq(W, B.QLORA_CODEBOOK_NF4, dq_format=B.QLORA_DQ_FP8_MEAN) if a.op == "quantize_fp8" else None
+    if a.op not in ("quantize", "quantize_fp8"):
         del W
     r = case.r
     X = A = Bm = dY = Y = None
@@ -58,6 +59,8 @@ def main(argv=None):
     def run():
         if a.op == "quantize":
             B.qlora_quantize_nf4_dq(W, out=w)
+        elif a.op == "quantize_fp8":
+            B.qlora_quantize_4bit_dq(W, B.QLORA_CODEBOOK_NF4, out=w8, dq_format=B.QLORA_DQ_FP8_MEAN)
         elif a.op == "dequant":
             B.qlora_dequant(w, out=out_w)
         elif a.op == "merge":
